@@ -1,0 +1,415 @@
+/*
+ * csa2_oracle.c -- plain CPU oracle for the CSA2 step over an FP4 main KV cache.
+ *
+ * TEST INFRASTRUCTURE: only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark use it. It is independent of the CUDA library (no shared
+ * code, tables or constants) and follows the definitions one step at a time in
+ * double precision. The page references and the readings taken where the pages
+ * are silent are listed in csa2_oracle.h.
+ */
+#include "csa2_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Number formats.                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* OCP 8-bit floating point, E4M3 variant: 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent field 0 is subnormal (2^-6 * m/8); the
+ * all-ones pattern S.1111.111 is NaN; there are no infinities. */
+double or_e4m3_value(uint8_t code) {
+    int sign = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Round to the nearest E4M3 value, ties to the code with an even mantissa,
+ * saturating to +-448 (the largest finite magnitude). */
+uint8_t or_e4m3_from_double(double x) {
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7E;
+    for (int c = 0; c < 126; ++c) {
+        double lo = or_e4m3_value((uint8_t)c);
+        double hi = or_e4m3_value((uint8_t)(c + 1));
+        if (a <= hi) {
+            double dlo = a - lo, dhi = hi - a;
+            int pick;
+            if (dlo < dhi) pick = c;
+            else if (dhi < dlo) pick = c + 1;
+            else pick = (c % 2 == 0) ? c : c + 1;
+            return sign | (uint8_t)pick;
+        }
+    }
+    return sign | 0x7E;
+}
+
+/* MX FP4 (E2M1): 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit;
+ * exponent field 0 is subnormal (0.5 * m). Grid: 0 0.5 1 1.5 2 3 4 6. */
+double or_e2m1_value(uint8_t code) {
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -v : v;
+}
+
+double or_bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+uint8_t or_e2m1_code(double x, double s) {
+    if (s == 0.0) return 0;
+    uint8_t sign = signbit(x) ? 0x8 : 0x0;
+    double a = fabs(x);
+    for (int c = 0; c < 7; ++c) {
+        double lo = or_e2m1_value((uint8_t)c) * s;
+        double hi = or_e2m1_value((uint8_t)(c + 1)) * s;
+        if (a <= hi) {
+            double dlo = a - lo, dhi = hi - a;
+            int pick;
+            if (dlo < dhi) pick = c;
+            else if (dhi < dlo) pick = c + 1;
+            else pick = (c % 2 == 0) ? c : c + 1;
+            return sign | (uint8_t)pick;
+        }
+    }
+    return sign | 0x7;
+}
+
+static double g_e4m3_table[256];
+static int g_e4m3_ready = 0;
+
+static void e4m3_table_init(void) {
+    if (g_e4m3_ready) return;
+    for (int i = 0; i < 256; ++i) g_e4m3_table[i] = or_e4m3_value((uint8_t)i);
+    g_e4m3_ready = 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP4 main KV: one E4M3 scale per channel per 64-entry block.               */
+/* ------------------------------------------------------------------------ */
+
+#define OR_BLOCK 64
+
+int or_fp4_kv_pack(const float* kv, int B, int N, int D,
+                   uint8_t* kv_packed, uint8_t* kv_scale) {
+    if (!kv || !kv_packed || !kv_scale || B < 0 || N < 0 || D <= 0) return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    int nblk = N / OR_BLOCK;
+    for (int b = 0; b < B; ++b) {
+        for (int blk = 0; blk < nblk; ++blk) {
+            for (int c = 0; c < D; ++c) {
+                double amax = 0.0;
+                for (int r = 0; r < OR_BLOCK; ++r) {
+                    int n = blk * OR_BLOCK + r;
+                    float x = kv[((size_t)b * N + n) * D + c];
+                    if (!isfinite(x)) return OR_NONFINITE;
+                    if (fabs((double)x) > amax) amax = fabs((double)x);
+                }
+                uint8_t sc = or_e4m3_from_double(amax / 6.0);
+                kv_scale[((size_t)b * nblk + blk) * D + c] = sc;
+                double s = or_e4m3_value(sc);
+                for (int r = 0; r < OR_BLOCK; ++r) {
+                    int n = blk * OR_BLOCK + r;
+                    float x = kv[((size_t)b * N + n) * D + c];
+                    uint8_t code = or_e2m1_code((double)x, s);
+                    uint8_t* byte = &kv_packed[((size_t)b * N + n) * (D / 2) + c / 2];
+                    if (c % 2 == 0)
+                        *byte = (uint8_t)((*byte & 0xF0) | code);
+                    else
+                        *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+                }
+            }
+        }
+    }
+    return OR_OK;
+}
+
+static double kv_value(const uint8_t* kv_packed, const uint8_t* kv_scale,
+                       int N, int D, int b, int n, int c) {
+    uint8_t byte = kv_packed[((size_t)b * N + n) * (D / 2) + c / 2];
+    uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    uint8_t sc = kv_scale[((size_t)b * (N / OR_BLOCK) + n / OR_BLOCK) * D + c];
+    return or_e2m1_value(code) * or_e4m3_value(sc);
+}
+
+int or_fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale,
+                     int B, int N, int D, double* out) {
+    if (!kv_packed || !kv_scale || !out || B < 0 || N < 0 || D <= 0) return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n)
+            for (int c = 0; c < D; ++c)
+                out[((size_t)b * N + n) * D + c] = kv_value(kv_packed, kv_scale, N, D, b, n, c);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Indexer score: s_j = sum_h w_h * ReLU(q_h . k_j).                          */
+/* ------------------------------------------------------------------------ */
+
+static double score_one(const uint8_t* q, const float* w, const uint8_t* k, int Hi, int Di) {
+    double s = 0.0;
+    for (int h = 0; h < Hi; ++h) {
+        double dot = 0.0;
+        for (int c = 0; c < Di; ++c)
+            dot += g_e4m3_table[q[(size_t)h * Di + c]] * g_e4m3_table[k[c]];
+        double relu = dot > 0.0 ? dot : 0.0;
+        s += (double)w[h] * relu;
+    }
+    return s;
+}
+
+int or_index_score(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                   int B, int Tq, int N, int Hi, int Di,
+                   const int32_t* nvalid, const int32_t* cand, int C,
+                   double* scores) {
+    if (!idx_q || !idx_w || !idx_k || !scores || B < 0 || Tq < 0 || N < 0 || Hi <= 0 || Di <= 0)
+        return OR_BAD_ARG;
+    if (!cand && !nvalid) return OR_BAD_ARG;
+    if (cand && C <= 0) return OR_BAD_ARG;
+    e4m3_table_init();
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < Tq; ++t) {
+            size_t row = (size_t)b * Tq + t;
+            const uint8_t* q = idx_q + row * Hi * Di;
+            const float* w = idx_w + row * Hi;
+            if (!cand) {
+                int nv = nvalid[row];
+                if (nv < 0 || nv > N) return OR_BAD_ARG;
+                for (int j = 0; j < N; ++j) {
+                    double* dst = &scores[row * N + j];
+                    if (j < nv)
+                        *dst = score_one(q, w, idx_k + ((size_t)b * N + j) * Di, Hi, Di);
+                    else
+                        *dst = -INFINITY;
+                }
+            } else {
+                for (int i = 0; i < C; ++i) {
+                    int j = cand[row * C + i];
+                    double* dst = &scores[row * C + i];
+                    if (j < 0) { *dst = -INFINITY; continue; }
+                    if (j >= N) return OR_BAD_INDEX;
+                    *dst = score_one(q, w, idx_k + ((size_t)b * N + j) * Di, Hi, Di);
+                }
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Top-K by (score descending, id ascending); output ascending by id.        */
+/* ------------------------------------------------------------------------ */
+
+typedef struct { double score; int32_t id; } scored_id;
+
+static int cmp_rank(const void* pa, const void* pb) {
+    const scored_id* a = (const scored_id*)pa;
+    const scored_id* b = (const scored_id*)pb;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->id < b->id) ? -1 : (a->id > b->id);
+}
+
+static int cmp_i32(const void* pa, const void* pb) {
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a < b) ? -1 : (a > b);
+}
+
+int or_topk(const double* scores, int rows, int ld,
+            const int32_t* nvalid, const int32_t* cand,
+            int K, int32_t* topk) {
+    if (!scores || !topk || rows < 0 || ld < 0 || K <= 0) return OR_BAD_ARG;
+    if (!cand && !nvalid) return OR_BAD_ARG;
+    scored_id* list = (scored_id*)malloc(sizeof(scored_id) * (size_t)(ld > 0 ? ld : 1));
+    int32_t* chosen = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+    if (!list || !chosen) { free(list); free(chosen); return OR_BAD_ARG; }
+    int rc = OR_OK;
+    for (int r = 0; r < rows && rc == OR_OK; ++r) {
+        int n = 0;
+        if (!cand) {
+            int nv = nvalid[r];
+            if (nv < 0 || nv > ld) { rc = OR_BAD_ARG; break; }
+            for (int j = 0; j < nv; ++j) {
+                list[n].score = scores[(size_t)r * ld + j];
+                list[n].id = j;
+                ++n;
+            }
+        } else {
+            for (int i = 0; i < ld; ++i) {
+                int32_t id = cand[(size_t)r * ld + i];
+                if (id < 0) continue;
+                list[n].score = scores[(size_t)r * ld + i];
+                list[n].id = id;
+                ++n;
+            }
+        }
+        for (int i = 0; i < n; ++i)
+            if (isnan(list[i].score)) { rc = OR_NONFINITE; break; }
+        if (rc != OR_OK) break;
+        qsort(list, (size_t)n, sizeof(scored_id), cmp_rank);
+        int m = n < K ? n : K;
+        for (int i = 0; i < m; ++i) chosen[i] = list[i].id;
+        qsort(chosen, (size_t)m, sizeof(int32_t), cmp_i32);
+        for (int i = 0; i < K; ++i) topk[(size_t)r * K + i] = (i < m) ? chosen[i] : -1;
+    }
+    free(list);
+    free(chosen);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sparse softmax attention over the selected rows; K doubles as V.          */
+/* ------------------------------------------------------------------------ */
+
+int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                   const int32_t* topk, int B, int Tq, int Hq, int D, int N, int K,
+                   double softmax_scale, double* out, double* lse) {
+    if (!q || !kv_packed || !kv_scale || !topk || !out || B < 0 || Tq < 0 || Hq <= 0 ||
+        D <= 0 || N < 0 || K <= 0)
+        return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    double* v = (double*)malloc(sizeof(double) * (size_t)K * D);
+    double* logit = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!v || !logit) { free(v); free(logit); return OR_BAD_ARG; }
+    int rc = OR_OK;
+    for (int b = 0; b < B && rc == OR_OK; ++b) {
+        for (int t = 0; t < Tq && rc == OR_OK; ++t) {
+            size_t row = (size_t)b * Tq + t;
+            /* dequantise the selected rows */
+            int n = 0;
+            for (int k = 0; k < K; ++k) {
+                int32_t id = topk[row * K + k];
+                if (id < 0) continue;
+                if (id >= N) { rc = OR_BAD_INDEX; break; }
+                for (int c = 0; c < D; ++c)
+                    v[(size_t)n * D + c] = kv_value(kv_packed, kv_scale, N, D, b, id, c);
+                ++n;
+            }
+            if (rc != OR_OK) break;
+            for (int h = 0; h < Hq; ++h) {
+                const uint16_t* qh = q + (row * Hq + h) * D;
+                double* oh = out + (row * Hq + h) * D;
+                if (n == 0) {
+                    for (int c = 0; c < D; ++c) oh[c] = 0.0;
+                    if (lse) lse[row * Hq + h] = -INFINITY;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int k = 0; k < n; ++k) {
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c) dot += or_bf16_value(qh[c]) * v[(size_t)k * D + c];
+                    logit[k] = softmax_scale * dot;
+                    if (logit[k] > m) m = logit[k];
+                }
+                double z = 0.0;
+                for (int k = 0; k < n; ++k) {
+                    logit[k] = exp(logit[k] - m); /* now the unnormalised weight */
+                    z += logit[k];
+                }
+                for (int c = 0; c < D; ++c) {
+                    double acc = 0.0;
+                    for (int k = 0; k < n; ++k) acc += logit[k] * v[(size_t)k * D + c];
+                    oh[c] = acc / z;
+                }
+                if (lse) lse[row * Hq + h] = m + log(z);
+            }
+        }
+    }
+    free(v);
+    free(logit);
+    return rc;
+}
+
+int or_dense_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                  const int32_t* nvalid, int B, int Tq, int Hq, int D, int N,
+                  double softmax_scale, double* out, double* lse) {
+    if (!q || !kv_packed || !kv_scale || !nvalid || !out || B < 0 || Tq < 0 || Hq <= 0 ||
+        D <= 0 || N < 0)
+        return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    double* p = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    if (!p) return OR_BAD_ARG;
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < Tq; ++t) {
+            size_t row = (size_t)b * Tq + t;
+            int nv = nvalid[row];
+            if (nv < 0 || nv > N) { free(p); return OR_BAD_ARG; }
+            for (int h = 0; h < Hq; ++h) {
+                const uint16_t* qh = q + (row * Hq + h) * D;
+                double* oh = out + (row * Hq + h) * D;
+                /* pass 1: logits and their maximum */
+                double m = -INFINITY;
+                for (int j = 0; j < nv; ++j) {
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c)
+                        dot += or_bf16_value(qh[c]) * kv_value(kv_packed, kv_scale, N, D, b, j, c);
+                    p[j] = softmax_scale * dot;
+                    if (p[j] > m) m = p[j];
+                }
+                /* pass 2: normalised probabilities and the weighted sum */
+                double z = 0.0;
+                for (int j = 0; j < nv; ++j) z += exp(p[j] - m);
+                for (int c = 0; c < D; ++c) oh[c] = 0.0;
+                for (int j = 0; j < nv; ++j) {
+                    double pj = exp(p[j] - m) / z;
+                    for (int c = 0; c < D; ++c)
+                        oh[c] += pj * kv_value(kv_packed, kv_scale, N, D, b, j, c);
+                }
+                if (lse) lse[row * Hq + h] = (nv > 0) ? m + log(z) : -INFINITY;
+            }
+        }
+    }
+    free(p);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One layer in FULL / REINDEX / REUSE mode.                                 */
+/* ------------------------------------------------------------------------ */
+
+int or_layer_step(int mode, const uint16_t* q, const uint8_t* idx_q, const float* idx_w,
+                  const uint8_t* idx_k, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                  const int32_t* nvalid, int B, int Tq, int N, int D, int Hq,
+                  int Hi, int Di, int K, int C, int use_pool, double softmax_scale,
+                  int32_t* topk_io, int32_t* cand_io, double* out, double* lse) {
+    int rows = B * Tq;
+    int rc;
+    if (!topk_io) return OR_BAD_ARG;
+    if (mode == OR_MODE_FULL || mode == OR_MODE_REINDEX) {
+        int pooled = (mode == OR_MODE_REINDEX) && use_pool;
+        if (pooled && (!cand_io || C <= 0)) return OR_BAD_ARG;
+        int ld = pooled ? C : N;
+        double* scores = (double*)malloc(sizeof(double) * (size_t)rows * (ld > 0 ? ld : 1));
+        if (!scores) return OR_BAD_ARG;
+        rc = or_index_score(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid,
+                            pooled ? cand_io : NULL, C, scores);
+        if (rc == OR_OK)
+            rc = or_topk(scores, rows, ld, pooled ? NULL : nvalid, pooled ? cand_io : NULL,
+                         K, topk_io);
+        if (rc == OR_OK && mode == OR_MODE_FULL && C > 0 && cand_io)
+            rc = or_topk(scores, rows, ld, nvalid, NULL, C, cand_io);
+        free(scores);
+        if (rc != OR_OK) return rc;
+    } else if (mode != OR_MODE_REUSE) {
+        return OR_BAD_ARG;
+    }
+    return or_sparse_attn(q, kv_packed, kv_scale, topk_io, B, Tq, Hq, D, N, K,
+                          softmax_scale, out, lse);
+}
