@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark: CSA2 decode layer step at 128K tokens of context (FULL mode).
+
+Workload "decode_128k_full": batch 32, one query token each, N = 32768 FP4
+main-KV entries of dim 512 (128K tokens at 4:1 compression), 64 bf16 query
+heads, indexer 64 heads x 128 with integer E4M3 values, top-2048, lengths
+uniform in [16384, 32768]. One step = one pass of the whole hot path over the
+batch: indexer scores -> top-K -> gather + FP4 dequant + sparse attention (+
+split combine). The FP4 cache is built once before timing (a cache is built
+when tokens arrive, not per step). Inputs are resident in HBM; L2 is flushed
+(256 MiB write) between timed steps, outside the timed events.
+
+Prints one JSON line. With --impl reference it times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s at 128K ctx; achieved HBM GB/s vs 8 TB/s peak"
+UNIT = "layer-steps/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_workload(w, rank: int):
+    """Weak scaling: every rank gets its own batch of sequences (its own seed)."""
+    return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# --------------------------------------------------------------- algorithmic bytes
+def algorithmic_bytes(w, nvalid: np.ndarray, topk: np.ndarray) -> dict:
+    """Bytes each kernel must move at least, from the realised lengths and the
+    selected indices (distinct 64-entry scale blocks per sequence)."""
+    rows = w.B * w.Tq
+    nv = nvalid.reshape(-1).astype(np.int64)
+    tk = topk.reshape(rows, w.K)
+    sel = (tk >= 0).sum(axis=1).astype(np.int64)
+    blocks = np.array([np.unique(r[r >= 0] // 64).size for r in tk], np.int64)
+    idx_k = int(nv.sum()) * w.Di
+    idx_qw = rows * (w.Hi * w.Di + 4 * w.Hi)
+    scores = int(nv.sum()) * 4
+    kv_rows = int(sel.sum()) * (w.D // 2)
+    scale_rows = int(blocks.sum()) * w.D
+    q_out = 2 * rows * w.Hq * w.D * 2
+    idx = rows * w.K * 4
+    return {
+        "score": idx_k + idx_qw + scores,
+        "topk": scores + idx,
+        "attn": kv_rows + scale_rows + q_out + idx,
+        "step": idx_k + idx_qw + kv_rows + scale_rows + q_out,
+        "flops_score": int(nv.sum()) * w.Hi * w.Di * 2,
+        "flops_attn": int(sel.sum()) * w.Hq * w.D * 4,
+    }
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from fp4_kv_cache_step_b200 import build as libbuild
+    from fp4_kv_cache_step_b200 import csa2
+    from fp4_kv_cache_step_b200 import workloads as wl
+    from fp4_kv_cache_step_b200.runner import DeviceWorkload
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        libbuild.build()
+    if world > 1:
+        dist.barrier()
+    csa2.load()
+
+    w = rank_workload(wl.CONFIGS[args.config], rank)
+    dw = DeviceWorkload(w, dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        dw.step()
+    csa2.check_device_errors()
+
+    # ---- timed steps (device events on the launching stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            ev[i][0].record(stream)
+            dw.step()
+            ev[i][1].record(stream)
+        barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    csa2.check_device_errors()
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ms_per_step = max_total_ms / args.steps
+    value = world * args.steps / (max_total_ms / 1e3)
+
+    # ---- per-kernel timing: the same kernels through the individual calls
+    nsplit_ws = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K)
+    kern = {"score": [], "topk": [], "attn": []}
+    scores = torch.empty((w.B, w.Tq, w.N), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(int(nsplit_ws), 256), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(dw.out[0])
+    lse = torch.empty_like(dw.lse[0])
+    for i in range(args.warmup + args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.fill_(i & 0xff)
+        evs[0].record(stream)
+        csa2.csa2_index_score(dw.idx_q[0], dw.idx_w[0], dw.idx_k, nvalid=dw.nvalid, out=scores)
+        evs[1].record(stream)
+        csa2.csa2_topk(scores, w.K, nvalid=dw.nvalid, out=dw.topk)
+        evs[2].record(stream)
+        flush.fill_(i & 0xff)
+        evs[3].record(stream)
+        csa2.csa2_sparse_attn(dw.q[0], dw.kv_packed, dw.kv_scale, dw.topk, w.softmax_scale,
+                              out=out, lse=lse, workspace=ws)
+        e4 = torch.cuda.Event(enable_timing=True)
+        e4.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            kern["score"].append(evs[0].elapsed_time(evs[1]))
+            kern["topk"].append(evs[1].elapsed_time(evs[2]))
+            kern["attn"].append(evs[3].elapsed_time(e4))
+    kern_us = {k: 1e3 * statistics.mean(v) for k, v in kern.items()}
+
+    nvalid = wl.nvalid(w)
+    ab = algorithmic_bytes(w, nvalid, dw.topk.cpu().numpy())
+    hbm_peak, tf_peak, peak_kind = measured_peaks()
+    dom = max(("score", "attn", "topk"), key=lambda k: kern_us[k])
+    if dom == "attn" and args.attn_bound == "tensor":
+        achieved = ab["flops_attn"] / (kern_us["attn"] * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": achieved / tf_peak}
+    else:
+        achieved = ab[dom] / (kern_us[dom] * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak}
+    roof.update({"kernel": dom, "peak_source": peak_kind + " (MEASURED_PEAKS.json)"
+                 if peak_kind == "measured" else "fallback", "traffic": args.traffic})
+
+    # ---- end to end through the C ABI with pinned host buffers
+    e2e = run_e2e(args, w, dw, flush, csa2, torch)
+
+    step_gbs = ab["step"] / (ms_per_step * 1e-3) / 1e9
+    launches_per_step = 3 + (1 if nsplit_ws > 0 else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Tq": w.Tq, "N": w.N, "D": w.D, "Hq": w.Hq,
+                   "Hi": w.Hi, "Di": w.Di, "K": w.K, "context_tokens": 4 * w.N,
+                   "kv_format": "E2M1 + E4M3 scale per channel per 64 entries",
+                   "arith": "indexer e4m3 x e4m3 -> f32; attention f16 x f16 -> f32; out bf16",
+                   "l2": "flushed between timed steps (256 MiB write outside the timed events)",
+                   "parallelism": "dp%d (independent batches per GPU)" % world},
+        "step_algorithmic_bytes": ab["step"],
+        "step_gbs": step_gbs, "step_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
+        "step_frac_of_measured_hbm": step_gbs / hbm_peak,
+        "query_tokens_per_s": value * w.B * w.Tq,
+        "kernel_us": kern_us,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample_rows)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, dw, flush, csa2, torch):
+    """Same step through the public call, with this step's query-side inputs
+    copied from pinned host memory and the outputs copied back, all inside the
+    timed region. The FP4 cache and indexer keys stay resident (they are the
+    cache)."""
+    from fp4_kv_cache_step_b200 import workloads as wl
+    stream = torch.cuda.current_stream()
+    host_in = {
+        "q": torch.from_numpy(wl.q(w, 0).view(np.int16)).view(torch.bfloat16).pin_memory(),
+        "idx_q": torch.from_numpy(wl.idx_q(w, 0)).pin_memory(),
+        "idx_w": torch.from_numpy(wl.idx_w(w, 0)).pin_memory(),
+        "nvalid": torch.from_numpy(wl.nvalid(w)).pin_memory(),
+    }
+    dev_in = {"q": dw.q[0], "idx_q": dw.idx_q[0], "idx_w": dw.idx_w[0], "nvalid": dw.nvalid}
+    host_out = torch.empty(dw.out[0].shape, dtype=torch.bfloat16).pin_memory()
+    host_lse = torch.empty(dw.lse[0].shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * 2 + host_lse.numel() * 4
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        dw.step(layers=[0])
+        host_out.copy_(dw.out[0], non_blocking=True)
+        host_lse.copy_(dw.lse[0], non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    return {"value": 1e3 / ms, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_layer_steps(w, rows):
+    """Time the oracle's FULL layer step on the given batch rows (cache build
+    excluded). Returns seconds."""
+    import oracle
+    from fp4_kv_cache_step_b200 import workloads as wl
+    nv_all = wl.nvalid(w)
+    total = 0.0
+    for b in rows:
+        packed, sc = oracle.fp4_kv_pack(wl.kv(w, rows=[b]))
+        ik = wl.idx_k(w, rows=[b])
+        q = wl.q(w, 0, rows=[b])
+        iq = wl.idx_q(w, 0, rows=[b])
+        iw = wl.idx_w(w, 0, rows=[b])
+        topk = np.full((1, w.Tq, w.K), -1, np.int32)
+        t0 = time.perf_counter()
+        oracle.layer_step(oracle.MODE_FULL, q, iq, iw, ik, packed, sc, nv_all[b:b + 1], w.K,
+                          w.softmax_scale, topk)
+        total += time.perf_counter() - t0
+    return total
+
+
+def cpu_baseline(w, nrows):
+    import oracle
+    oracle.build()
+    rows = list(range(min(nrows, w.B)))
+    secs = oracle_layer_steps(w, rows)
+    per_step = secs * w.B / len(rows)
+    return {"value": 1.0 / per_step, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d of %d sequences of one FULL layer step (score + top-K + attention, "
+                      "cache build excluded), single-threaded fp64; scaled to a %d-sequence "
+                      "layer step" % (len(rows), w.B, w.B)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    sys.path.insert(0, ROOT)
+    from fp4_kv_cache_step_b200 import workloads as wl
+    import oracle
+    oracle.build()
+    w = wl.CONFIGS[args.config]
+    for i in range(args.warmup):
+        oracle_layer_steps(w, [i % w.B])
+    secs = [oracle_layer_steps(w, [i % w.B]) for i in range(args.steps)]
+    per_step = statistics.mean(secs) * w.B
+    value = 1.0 / per_step
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "Tq": w.Tq, "N": w.N, "D": w.D, "Hq": w.Hq,
+                       "Hi": w.Hi, "Di": w.Di, "K": w.K, "context_tokens": 4 * w.N,
+                       "parallelism": "none (CPU oracle, rank 0)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "each step: one sequence of the %d-sequence FULL layer "
+                                       "step, scaled by %d; single-threaded fp64" % (w.B, w.B)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--cpu-sample-rows", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn-bound", default="tensor", choices=["tensor", "hbm"])
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if captured")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

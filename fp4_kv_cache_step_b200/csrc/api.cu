@@ -1,0 +1,295 @@
+// api.cu -- the exported C ABI of libcsa2_fp4 (declared in include/csa2.h):
+// argument checks, the per-device error word, workspace planning and the
+// FULL / REINDEX / REUSE layer-step dispatcher.
+//
+// Modes: "Detailed Notes On DeepSeek V4 Point 1 Flash In Simple Words",
+// section "The Three Modes Full Reindex And Reuse", and the mengman.github.io
+// interpretation, section 3.3 (mode table) and 3.4 (hierarchical indexer):
+// FULL indexes for itself; REINDEX reuses the main KV and indexer keys but
+// scores with its own indexer query, optionally only inside the candidate pool
+// the first FULL layer kept; REUSE takes the latest top-K unchanged. The modes
+// only choose which kernels run; the shared buffers are passed by pointer.
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// First device-side data error per device (0 = none).
+__device__ int g_device_error;
+
+csa2_status fail(csa2_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+csa2_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(CSA2_ERR_CUDA, "%s: CUDA error %d (%s)", where, (int)e, cudaGetErrorString(e));
+}
+
+csa2_status ok() {
+  g_last_error.clear();
+  return CSA2_OK;
+}
+
+int* device_error_word(cudaError_t* e_out) {
+  static std::mutex mu;
+  static int* words[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 128) {
+    *e_out = e != cudaSuccess ? e : cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!words[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) {
+      *e_out = e;
+      return nullptr;
+    }
+    words[dev] = static_cast<int*>(p);
+  }
+  *e_out = cudaSuccess;
+  return words[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+#define CHECK_ARG(cond, ...) \
+  do {                        \
+    if (!(cond)) return fail(CSA2_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define CHECK_PTR(p) CHECK_ARG((p) != nullptr && aligned16(p), "%s must be a non-null 16-byte aligned device pointer", #p)
+
+csa2_status check_kv(const void* kv_packed, const void* kv_scale, int B, int N, int D) {
+  CHECK_PTR(kv_packed);
+  CHECK_PTR(kv_scale);
+  CHECK_ARG(B >= 0 && N >= 0, "B=%d and N=%d must be >= 0", B, N);
+  CHECK_ARG(N % csa2::kBlockEntries == 0, "N=%d must be a multiple of 64", N);
+  CHECK_ARG(D > 0 && D % 32 == 0, "D=%d must be a positive multiple of 32", D);
+  return CSA2_OK;
+}
+
+csa2_status check_score_args(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                             int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
+                             const int32_t* cand, int C) {
+  CHECK_PTR(idx_q);
+  CHECK_PTR(idx_w);
+  CHECK_PTR(idx_k);
+  CHECK_ARG(B >= 0 && Tq >= 0 && N >= 0, "B, Tq, N must be >= 0");
+  CHECK_ARG(B <= 65535 && Tq <= 65535, "B=%d and Tq=%d must be <= 65535", B, Tq);
+  CHECK_ARG(Hi >= 1 && Hi <= 128, "Hi=%d must be in [1, 128]", Hi);
+  CHECK_ARG(Di >= 16 && Di <= 256 && Di % 16 == 0, "Di=%d must be a multiple of 16 in [16, 256]", Di);
+  if (cand) {
+    CHECK_PTR(cand);
+    CHECK_ARG(C >= 1, "C=%d must be >= 1 with a candidate pool", C);
+  } else {
+    CHECK_PTR(nvalid);
+  }
+  return CSA2_OK;
+}
+
+csa2_status check_attn_args(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                            const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N, int K,
+                            const uint16_t* out, const float* lse) {
+  csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
+  if (s != CSA2_OK) return s;
+  CHECK_PTR(q);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(out);
+  if (lse) CHECK_ARG(((uintptr_t)lse & 3u) == 0, "lse must be 4-byte aligned");
+  CHECK_ARG(Tq >= 0, "Tq=%d must be >= 0", Tq);
+  CHECK_ARG(Hq >= 1 && Hq <= 65535, "Hq=%d must be in [1, 65535]", Hq);
+  CHECK_ARG(K >= 1, "K=%d must be >= 1", K);
+  if (D != csa2::kHeadDim)
+    return fail(CSA2_ERR_UNSUPPORTED, "attention is built for D=512 only (got D=%d)", D);
+  return CSA2_OK;
+}
+
+size_t layer_scores_bytes(const csa2_layer_args* a, csa2_mode mode, const csa2_shared_state* st) {
+  if (mode == CSA2_MODE_REUSE) return 0;
+  const bool pooled = mode == CSA2_MODE_REINDEX && a->use_pool;
+  const size_t ld = pooled ? (size_t)st->C : (size_t)a->N;
+  return round_up((size_t)a->B * a->Tq * ld * sizeof(float));
+}
+
+}  // namespace
+
+extern "C" {
+
+csa2_status fp4_kv_pack(const float* kv, int B, int N, int D, uint8_t* kv_packed,
+                        uint8_t* kv_scale, csa2_stream_t stream) {
+  CHECK_PTR(kv);
+  csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
+  if (s != CSA2_OK) return s;
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "fp4_kv_pack");
+  e = csa2::launch_fp4_pack(kv, B, N, D, kv_packed, kv_scale, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_pack launch");
+  return ok();
+}
+
+csa2_status fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale, int B, int N, int D,
+                          float* out, csa2_stream_t stream) {
+  CHECK_PTR(out);
+  csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
+  if (s != CSA2_OK) return s;
+  cudaError_t e = csa2::launch_fp4_unpack(kv_packed, kv_scale, B, N, D, out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack launch");
+  return ok();
+}
+
+csa2_status csa2_index_score(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                             int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
+                             const int32_t* cand, int C, float* scores, csa2_stream_t stream) {
+  CHECK_PTR(scores);
+  csa2_status s = check_score_args(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid, cand, C);
+  if (s != CSA2_OK) return s;
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_index_score");
+  e = csa2::launch_index_score(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid, cand, cand ? C : 0,
+                               scores, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_index_score launch");
+  return ok();
+}
+
+csa2_status csa2_topk(const float* scores, int ld, const int32_t* nvalid, const int32_t* cand,
+                      int B, int Tq, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
+                      csa2_stream_t stream) {
+  CHECK_PTR(scores);
+  CHECK_PTR(topk_idx);
+  CHECK_ARG(B >= 0 && Tq >= 0, "B=%d and Tq=%d must be >= 0", B, Tq);
+  CHECK_ARG(ld >= 0 && ld <= (1 << 30), "ld=%d must be in [0, 2^30]", ld);
+  CHECK_ARG(K >= 1 && K <= 65536, "K=%d must be in [1, 65536]", K);
+  if (cand) CHECK_PTR(cand); else CHECK_PTR(nvalid);
+  if (cand_out) {
+    CHECK_PTR(cand_out);
+    CHECK_ARG(Cout >= 1 && Cout <= 65536, "Cout=%d must be in [1, 65536]", Cout);
+  }
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_topk");
+  e = csa2::launch_topk(scores, ld, cand ? nullptr : nvalid, cand, B * Tq, K, topk_idx,
+                        cand_out ? Cout : 0, cand_out, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_topk launch");
+  return ok();
+}
+
+size_t csa2_sparse_attn_workspace_bytes(int B, int Tq, int Hq, int D, int K) {
+  (void)D;
+  if (B <= 0 || Tq <= 0 || Hq <= 0 || K <= 0) return 0;
+  return round_up(csa2::sparse_attn_workspace_bytes(B, Tq, Hq, K));
+}
+
+csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                             const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N, int K,
+                             float softmax_scale, uint16_t* out, float* lse, void* workspace,
+                             size_t workspace_bytes, csa2_stream_t stream) {
+  csa2_status s = check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
+  if (s != CSA2_OK) return s;
+  const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn needs %zu workspace bytes (got %zu)", need,
+                workspace_bytes);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_sparse_attn");
+  e = csa2::launch_sparse_attn(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, N, K, softmax_scale,
+                               out, lse, workspace, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_sparse_attn launch");
+  return ok();
+}
+
+size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* a, csa2_mode mode,
+                                       const csa2_shared_state* st) {
+  if (!a || !st) return 0;
+  return layer_scores_bytes(a, mode, st) +
+         csa2_sparse_attn_workspace_bytes(a->B, a->Tq, a->Hq, a->D, a->K);
+}
+
+csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_shared_state* st,
+                            void* workspace, size_t workspace_bytes, csa2_stream_t stream) {
+  CHECK_ARG(a != nullptr && st != nullptr, "args and shared state must be non-null");
+  CHECK_ARG(mode == CSA2_MODE_FULL || mode == CSA2_MODE_REINDEX || mode == CSA2_MODE_REUSE,
+            "unknown mode %d", (int)mode);
+  csa2_status s = check_attn_args(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq,
+                                  a->Hq, a->D, a->N, a->K, a->out, a->lse);
+  if (s != CSA2_OK) return s;
+  const bool pooled = mode == CSA2_MODE_REINDEX && a->use_pool;
+  const bool emit = mode == CSA2_MODE_FULL && a->emit_pool;
+  if (mode != CSA2_MODE_REUSE) {
+    s = check_score_args(a->idx_q, a->idx_w, st->idx_k, a->B, a->Tq, a->N, a->Hi, a->Di, a->nvalid,
+                         pooled ? st->cand_idx : nullptr, st->C);
+    if (s != CSA2_OK) return s;
+    CHECK_PTR(a->nvalid);
+    if (pooled || emit) {
+      CHECK_PTR(st->cand_idx);
+      CHECK_ARG(st->C >= 1 && st->C <= 65536, "pool size C=%d must be in [1, 65536]", st->C);
+    }
+    if (emit) CHECK_ARG(st->C >= a->K, "pool size C=%d must be >= K=%d", st->C, a->K);
+  }
+  const size_t need = csa2_layer_step_workspace_bytes(a, mode, st);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA2_ERR_WORKSPACE, "csa2_layer_step needs %zu workspace bytes (got %zu)", need,
+                workspace_bytes);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_layer_step");
+  cudaStream_t cs = (cudaStream_t)stream;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const size_t scores_bytes = layer_scores_bytes(a, mode, st);
+  if (mode != CSA2_MODE_REUSE) {
+    float* scores = reinterpret_cast<float*>(ws);
+    const int ld = pooled ? st->C : a->N;
+    e = csa2::launch_index_score(a->idx_q, a->idx_w, st->idx_k, a->B, a->Tq, a->N, a->Hi, a->Di,
+                                 a->nvalid, pooled ? st->cand_idx : nullptr, pooled ? st->C : 0,
+                                 scores, err, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step score");
+    e = csa2::launch_topk(scores, ld, pooled ? nullptr : a->nvalid, pooled ? st->cand_idx : nullptr,
+                          a->B * a->Tq, a->K, st->topk_idx, emit ? st->C : 0,
+                          emit ? st->cand_idx : nullptr, err, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step top-k");
+  }
+  e = csa2::launch_sparse_attn(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq, a->Hq,
+                               a->N, a->K, a->softmax_scale, a->out, a->lse,
+                               ws ? ws + scores_bytes : nullptr, err, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step attention");
+  return ok();
+}
+
+csa2_status csa2_check_device_errors(csa2_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_check_device_errors sync");
+  int code = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&code, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_check_device_errors read");
+  if (code != 0) {
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "csa2_check_device_errors clear");
+    return fail((csa2_status)code, "device reported error code %d", code);
+  }
+  return ok();
+}
+
+const char* csa2_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

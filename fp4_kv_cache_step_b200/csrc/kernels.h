@@ -1,0 +1,33 @@
+// kernels.h -- internal launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa2 {
+
+cudaError_t launch_fp4_pack(const float* kv, int B, int N, int D, uint8_t* packed,
+                            uint8_t* scale, int* err, cudaStream_t stream);
+cudaError_t launch_fp4_unpack(const uint8_t* packed, const uint8_t* scale, int B, int N, int D,
+                              float* out, cudaStream_t stream);
+
+// Indexer scores; see csa2_index_score for the contract.
+cudaError_t launch_index_score(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                               int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
+                               const int32_t* cand, int C, float* scores, int* err,
+                               cudaStream_t stream);
+
+// Top-K (and optional second, larger selection) per row; see csa2_topk.
+cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, const int32_t* cand,
+                        int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
+                        int* err, cudaStream_t stream);
+
+// Sparse attention; see csa2_sparse_attn.
+size_t sparse_attn_workspace_bytes(int B, int Tq, int Hq, int K);
+cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
+                               const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
+                               int Hq, int N, int K, float softmax_scale, uint16_t* out,
+                               float* lse, void* workspace, int* err, cudaStream_t stream);
+
+}  // namespace csa2

@@ -1,0 +1,230 @@
+/*
+ * csa2.h -- C ABI of libcsa2_fp4: the CSA2 attention step over an FP4 main KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * What the step computes follows two of the pages that describe
+ * DeepSeek-V4.1-Flash:
+ *   [N] "Detailed Notes On DeepSeek V4 Point 1 Flash In Simple Words"
+ *       (personal-website-enc.pages.dev), sections "Compressed Sparse
+ *       Attention 2 Or CSA2 In Simple Terms", "The Three Modes Full Reindex And
+ *       Reuse", "Hierarchical Sparse Indexer In Simple Terms", "FP4 Main KV
+ *       Cache To Halve Storage Again";
+ *   [M] "DeepSeek-V4.1-Flash tech-report interpretation" (mengman.github.io),
+ *       section 3.3 (CSA2, its three static modes), 3.4 (hierarchical sparse
+ *       indexer) and 3.5 (FP4 main KV cache).
+ * A layer's indexer scores past main-KV entries against the current query and
+ * keeps the top-K; attention then runs over only those entries, which are
+ * stored as E2M1 values with E4M3 scales and dequantised before attention.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless stated; the caller owns every buffer.
+ *    The library allocates no device memory; scratch comes from the caller's
+ *    workspace (size from the matching *_workspace_bytes query).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). Host-side argument errors are reported before anything is
+ *    launched; nothing is thrown across the ABI.
+ *  - Device-side data errors (an index outside [-1, N), a non-finite value, an
+ *    unsorted candidate list) do not trap: the kernel skips the bad element and
+ *    records the first error code in a per-device word that
+ *    csa2_check_device_errors() returns and clears.
+ *  - Layouts are row-major and contiguous. bf16 values are passed as their
+ *    16-bit patterns (uint16_t), E4M3 values as bytes.
+ *  - Packed FP4: byte c/2 of an entry holds channel c, low nibble = even c.
+ *    Scales: one E4M3 byte per channel per 64-entry block,
+ *    kv_scale[b][n/64][c] (this block-scale layout is the one the benchmark
+ *    configurations state; the pages' own 16-channel grouping is not built).
+ *  - Pointers must be 16-byte aligned; D must be 512 for attention; N must be a
+ *    multiple of 64.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* csa2_stream_t;
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or mode */
+  CSA2_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. D != 512) */
+  CSA2_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  CSA2_ERR_DEVICE_INDEX = 4,  /* device saw an index outside its range or an unsorted pool */
+  CSA2_ERR_NONFINITE = 5,     /* device saw a NaN or infinity where a finite value is needed */
+  CSA2_ERR_TIMEOUT = 6,       /* a bounded device wait ran out */
+  CSA2_ERR_WORKSPACE = 7      /* workspace pointer NULL or smaller than required */
+} csa2_status;
+
+/* The three static per-layer modes ([N] "The Three Modes Full Reindex And
+ * Reuse"; [M] 3.3): FULL scores its own indexer query against the shared
+ * indexer keys and picks fresh top-K; REINDEX reuses the main KV and indexer
+ * keys of an earlier FULL layer but scores with its own indexer query
+ * (optionally only inside the candidate pool, [M] 3.4); REUSE attends over the
+ * latest top-K indices with no indexing at all. */
+typedef enum {
+  CSA2_MODE_FULL = 0,
+  CSA2_MODE_REINDEX = 1,
+  CSA2_MODE_REUSE = 2
+} csa2_mode;
+
+/* ------------------------------------------------------------------------
+ * fp4_kv_pack -- quantise the main KV cache to E2M1 with E4M3 block scales
+ * ([N] "FP4 Main KV Cache To Halve Storage Again"; [M] 3.5: E2M1 values,
+ * E4M3 scales, no second-level global scale).
+ *
+ * For each (b, 64-entry block, channel c): amax = max |kv| over the block;
+ * scale = round-to-nearest-even E4M3 of amax / 6 (saturating at 448); each
+ * value gets the E2M1 code nearest to x / scale, ties to the even code,
+ * saturating at +-6, sign from x (scale 0 gives code 0).
+ *   kv         float   [B][N][D]      input, finite
+ *   kv_packed  uint8   [B][N][D/2]    output
+ *   kv_scale   uint8   [B][N/64][D]   output, E4M3
+ * Requires N % 64 == 0, D % 32 == 0. A NaN or infinity in kv records
+ * CSA2_ERR_NONFINITE on the device (its block is still written).
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status fp4_kv_pack(const float* kv, int B, int N, int D,
+                        uint8_t* kv_packed, uint8_t* kv_scale, csa2_stream_t stream);
+
+/* fp4_kv_unpack -- exact dequantisation: out[b][n][c] = e2m1(code) * e4m3(scale).
+ *   out        float   [B][N][D]      output (every value is exact in fp32) */
+CSA2_API csa2_status fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale,
+                          int B, int N, int D, float* out, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_index_score -- indexer scores ([N] "Compressed Sparse Attention 2 Or
+ * CSA2 In Simple Terms": each layer's small indexer scores which past entries
+ * are most relevant to the current query; the indexer keys are one shared key
+ * per entry).  Score of entry j for query (b, t):
+ *     s = sum_h idx_w[b][t][h] * max(0, sum_c idx_q[b][t][h][c] * idx_k[b][j][c])
+ * with E4M3 inputs and fp32 accumulation (exact for integer-valued inputs
+ * whose score magnitude stays below 2^24).
+ *   idx_q   uint8 [B][Tq][Hi][Di]  E4M3
+ *   idx_w   float [B][Tq][Hi]
+ *   idx_k   uint8 [B][N][Di]       E4M3, shared by all indexing layers
+ *   nvalid  int32 [B][Tq]          entries [0, nvalid) are visible (causal mask)
+ *   cand    int32 [B][Tq][C]       NULL for a full scan; otherwise the candidate
+ *                                  pool ([M] 3.4): ascending entry ids then -1
+ *   scores  float [B][Tq][N]       full scan: written for j < nvalid, the rest
+ *                                  of the row is not written;
+ *           float [B][Tq][C]       pool: score of cand[i], -inf where cand[i] < 0
+ * Requires Di % 16 == 0, Di <= 256, Hi <= 128.
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status csa2_index_score(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                             int B, int Tq, int N, int Hi, int Di,
+                             const int32_t* nvalid, const int32_t* cand, int C,
+                             float* scores, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_topk -- top-K selection ([N] CSA2 section: the indexer picks the top
+ * entries to attend to; [M] 3.3). Entries are ranked by (score descending,
+ * entry id ascending) -- the lower index wins a tie, and -0 equals +0 -- and
+ * the selected ids are written ascending, padded with -1 when fewer than K
+ * entries are valid.
+ *   scores   float [B][Tq][ld]
+ *   nvalid   int32 [B][Tq]     full scan: entries j < nvalid, id = j (cand NULL)
+ *   cand     int32 [B][Tq][ld] pool: entry i has id cand[i], skipped when < 0;
+ *                              ids must be ascending (checked on the device)
+ *   topk_idx int32 [B][Tq][K]  output
+ *   cand_out int32 [B][Tq][Cout] optional second selection with the same
+ *                              ranking (the hierarchical pool, [M] 3.4); the
+ *                              top-K is a subset of it. NULL to skip.
+ * Requires 1 <= K, Cout <= 65536 and ld <= 2^30. A NaN score records
+ * CSA2_ERR_NONFINITE.
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status csa2_topk(const float* scores, int ld, const int32_t* nvalid, const int32_t* cand,
+                      int B, int Tq, int K, int32_t* topk_idx,
+                      int Cout, int32_t* cand_out, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_sparse_attn -- gather + FP4 dequantisation + softmax attention over
+ * the selected entries only ([N] CSA2 section and "FP4 Main KV Cache To Halve
+ * Storage Again": values are dequantised back before attention). One shared
+ * main-KV head of dimension D serves as both key and value:
+ *     l_k = softmax_scale * q[b][t][h] . v_k,   v_k = dequant(kv row idx_k)
+ *     out[b][t][h] = sum_k softmax(l)_k v_k,     lse[b][t][h] = log sum_k e^{l_k}
+ * over the entries topk_idx[b][t][*] >= 0 (-1 is skipped; no valid entry gives
+ * out = 0 and lse = -inf). Accumulation is fp32; the output is rounded to bf16.
+ *   q         uint16 [B][Tq][Hq][D]  bf16
+ *   kv_packed uint8  [B][N][D/2],  kv_scale uint8 [B][N/64][D]
+ *   topk_idx  int32  [B][Tq][K]      ids in [-1, N); out-of-range ids are
+ *                                    skipped and recorded
+ *   out       uint16 [B][Tq][Hq][D]  bf16
+ *   lse       float  [B][Tq][Hq]     optional (NULL to skip), natural log
+ *   workspace device scratch of csa2_sparse_attn_workspace_bytes() bytes
+ * Requires D == 512, 1 <= Hq <= 65535, K >= 1.
+ * ------------------------------------------------------------------------ */
+CSA2_API size_t csa2_sparse_attn_workspace_bytes(int B, int Tq, int Hq, int D, int K);
+
+CSA2_API csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                             const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N, int K,
+                             float softmax_scale, uint16_t* out, float* lse,
+                             void* workspace, size_t workspace_bytes, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * csa2_layer_step -- one CSA2 layer in its static mode ([N] "The Three Modes
+ * Full Reindex And Reuse"; [M] 3.3, 3.4). The shared state holds non-owning
+ * device pointers that several layers pass to each other without copies: the
+ * main KV and indexer keys built by a FULL layer, and the latest top-K indices
+ * (and candidate pool) that REINDEX/REUSE layers consume.
+ *   FULL    : score [0, nvalid) -> top-K into st->topk_idx (and the top-C pool
+ *             into st->cand_idx when args->emit_pool and st->C > 0) -> attention
+ *   REINDEX : score [0, nvalid), or only st->cand_idx when args->use_pool,
+ *             with this layer's own indexer query -> top-K into st->topk_idx
+ *             -> attention
+ *   REUSE   : attention over st->topk_idx as it stands
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const uint8_t* kv_packed;   /* [B][N][D/2] */
+  const uint8_t* kv_scale;    /* [B][N/64][D] */
+  const uint8_t* idx_k;       /* [B][N][Di] E4M3; may be NULL when only REUSE runs */
+  int32_t* topk_idx;          /* [B][Tq][K]: written by FULL/REINDEX, read by all */
+  int32_t* cand_idx;          /* [B][Tq][C]: written by FULL (emit_pool), read by REINDEX (use_pool) */
+  int C;                      /* candidate pool size (0 = no pool) */
+} csa2_shared_state;
+
+typedef struct {
+  int B, Tq, N, D, Hq, Hi, Di, K;
+  const int32_t* nvalid;      /* [B][Tq] */
+  const uint16_t* q;          /* [B][Tq][Hq][D] bf16 attention query of this layer */
+  const uint8_t* idx_q;       /* [B][Tq][Hi][Di] E4M3 indexer query (FULL/REINDEX) */
+  const float* idx_w;         /* [B][Tq][Hi] indexer head weights (FULL/REINDEX) */
+  float softmax_scale;
+  uint16_t* out;              /* [B][Tq][Hq][D] bf16 */
+  float* lse;                 /* [B][Tq][Hq] or NULL */
+  int emit_pool;              /* FULL: also write the top-C pool into st->cand_idx */
+  int use_pool;               /* REINDEX: score only st->cand_idx */
+} csa2_layer_args;
+
+CSA2_API size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* args, csa2_mode mode,
+                                       const csa2_shared_state* st);
+
+CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* args, csa2_mode mode, csa2_shared_state* st,
+                            void* workspace, size_t workspace_bytes, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Errors.
+ * csa2_check_device_errors: synchronises `stream`, returns the first device
+ * data error recorded on the current device since the last check (CSA2_OK if
+ * none) and clears it.
+ * csa2_last_error: thread-local text for the last non-OK status returned on
+ * this thread (empty string if none). The pointer stays valid until the next
+ * call on the same thread.
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status csa2_check_device_errors(csa2_stream_t stream);
+CSA2_API const char* csa2_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */
