@@ -18,6 +18,12 @@ cudaError_t launch_index_score(const uint8_t* idx_q, const float* idx_w, const u
                                const int32_t* cand, int C, float* scores, int* err,
                                cudaStream_t stream);
 
+// Tensor-core scorer (score_tc.cu): full scans with Hi in {64, 128}, Di in {64, 128}.
+bool index_score_tc_supported(int B, int Tq, int Hi, int Di, const int32_t* cand);
+cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                                  int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
+                                  float* scores, int* err, cudaStream_t stream);
+
 // Top-K (and optional second, larger selection) per row; see csa2_topk.
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, const int32_t* cand,
                         int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,

@@ -9,10 +9,11 @@
 // interpretation, section 3.4: a REINDEX layer can score only inside the
 // candidate pool of the first FULL layer.
 //
-// This file holds the CUDA-core scorer: one CTA per (query row, 128 entries),
-// the query decoded once into shared memory (broadcast reads), each thread one
-// entry, heads in groups of 32 register accumulators. It serves the
-// candidate-pool gather and any shape the tensor-core scorer does not take.
+// This file holds the dispatcher and the CUDA-core scorer: one CTA per (query
+// row, 128 entries), the query decoded once into shared memory (broadcast
+// reads), each thread one entry, heads in groups of 32 register accumulators.
+// The CUDA-core scorer serves the candidate-pool gather and shapes the
+// tensor-core scorer (score_tc.cu) does not take.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -109,6 +110,9 @@ cudaError_t launch_index_score(const uint8_t* idx_q, const float* idx_w, const u
                                const int32_t* cand, int C, float* scores, int* err,
                                cudaStream_t stream) {
   if (B == 0 || Tq == 0) return cudaSuccess;
+  if (index_score_tc_supported(B, Tq, Hi, Di, cand))
+    return launch_index_score_tc(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid, scores, err,
+                                 stream);
   const int len = cand ? C : N;
   if (len == 0) return cudaSuccess;
   const size_t smem = ((size_t)Hi * Di + Hi) * sizeof(float);

@@ -1,0 +1,338 @@
+// score_tc.cu -- CSA2 indexer scoring on the 5th-generation tensor cores.
+//
+// "Detailed Notes On DeepSeek V4 Point 1 Flash In Simple Words", section
+// "Compressed Sparse Attention 2 Or CSA2 In Simple Terms": every indexing layer
+// scores all visible entries against its query; the keys are one shared
+// indexer key per entry. Score of entry j for query (b, t):
+//     s_j = sum_h w_h * max(0, q_h . k_j)
+//
+// Per (b, group of nq consecutive queries) the dot products form a dense
+// contraction D[j][(t, h)] = sum_c K[j][c] Q[(t, h)][c] with E4M3 operands and
+// fp32 accumulation: M = 128 entries (TMEM lanes), N = nq * Hi (TMEM columns),
+// K = Di. The kernel is persistent (one CTA per SM, a contiguous share of all
+// (group, 128-entry) tiles) and warp-specialised:
+//   warp 0     TMA producer: indexer-key tiles (128 x Di bytes, 128/64-byte
+//              swizzle) into a ring of shared-memory stages, and the group's
+//              query block (N x Di) into one of two query buffers;
+//   warp 1     allocates TMEM and issues tcgen05.mma kind::f8f6f4 (one thread),
+//              committing each tile to "stage free" and "accumulator full";
+//   warps 2-9  two epilogue warpgroups taking alternate tiles: TMEM -> registers,
+//              ReLU, head-weighted sum, masked store of the score.
+// Decode (nq = 1) streams the keys once at HBM rate; the tensor core is ~1/5
+// busy. Prefill chunks (nq = 256 / Hi) make it a real dense FP8 contraction.
+// Every mbarrier wait is bounded; a timeout is reported as CSA2_ERR_TIMEOUT.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa2 {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;
+constexpr int kThreads = 320;
+constexpr int kMaxGroups = 8192;
+
+struct TcParams {
+  int Tq, N, Hi, Di, nq, G, groups_per_b, stages;
+  uint32_t ncols;
+  const int32_t* nvalid;
+  const float* idx_w;
+  float* scores;
+  int* err;
+};
+
+__device__ __forceinline__ int group_tiles(const TcParams& p, int g) {
+  const int b = g / p.groups_per_b;
+  const int t0 = (g % p.groups_per_b) * p.nq;
+  int nmax = 0;
+  for (int t = t0; t < min(t0 + p.nq, p.Tq); ++t)
+    nmax = max(nmax, min(p.N, max(0, p.nvalid[(size_t)b * p.Tq + t])));
+  return (nmax + kTileM - 1) / kTileM;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap qmap, const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int tile_bytes = kTileM * p.Di;
+  const int n_mma = p.Hi * p.nq;
+  const int q_bytes = n_mma * p.Di;
+  uint8_t* kbuf = base;
+  uint8_t* qbuf = kbuf + p.stages * tile_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(qbuf + 2 * q_bytes);
+  uint64_t* empty = full + p.stages;
+  uint64_t* acc_full = empty + p.stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* q_full = acc_empty + 2;
+  uint64_t* q_empty = q_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* tile_pre = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));   // [G + 1]
+  int* scan_tmp = tile_pre + p.G + 1;                                               // [kThreads/32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- prefix of tile counts over groups (contiguous chunk per thread)
+  {
+    const int per = (p.G + kThreads - 1) / kThreads;
+    const int g0 = min(p.G, (int)threadIdx.x * per), g1 = min(p.G, g0 + per);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int c = group_tiles(p, g);
+      tile_pre[g + 1] = c;
+      local += c;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) scan_tmp[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w2 = 0; w2 < warp; ++w2) before += scan_tmp[w2];
+    int run = before + incl - local;
+    if (threadIdx.x == 0) tile_pre[0] = 0;
+    for (int g = g0; g < g1; ++g) {
+      run += tile_pre[g + 1];
+      tile_pre[g + 1] = run;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, p.ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const long long T = tile_pre[p.G];
+  const int lo = (int)(T * blockIdx.x / gridDim.x);
+  const int hi = (int)(T * (blockIdx.x + 1) / gridDim.x);
+  // first group whose tile range contains `lo`
+  int g_first = 0;
+  {
+    int a = 0, bnd = p.G;   // find largest g with tile_pre[g] <= lo
+    while (a < bnd) {
+      int m = (a + bnd + 1) >> 1;
+      if (tile_pre[m] <= lo) a = m; else bnd = m - 1;
+    }
+    g_first = min(a, max(p.G - 1, 0));
+  }
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int qseq = -1, cur_g = -1, g = g_first;
+      for (int tile = lo; tile < hi; ++tile) {
+        while (tile >= tile_pre[g + 1]) ++g;
+        const int b = g / p.groups_per_b;
+        if (g != cur_g) {
+          ++qseq;
+          const int qb = qseq & 1;
+          if (!mbar_wait(&q_empty[qb], ((qseq >> 1) & 1) ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&q_full[qb], q_bytes);
+          const int qrow = (b * p.Tq + (g % p.groups_per_b) * p.nq) * p.Hi;
+          tma_load_2d(&qmap, &q_full[qb], qbuf + qb * q_bytes, 0, qrow);
+          cur_g = g;
+        }
+        const int e = tile - tile_pre[g];
+        if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[stage], tile_bytes);
+        tma_load_2d(&kmap, &full[stage], kbuf + stage * tile_bytes, 0, b * p.N + e * kTileM);
+        if (++stage == p.stages) { stage = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_e4m3_f32(kTileM, n_mma);
+      int stage = 0;
+      uint32_t ph = 0;
+      int qseq = -1, cur_g = -1, g = g_first, k = 0;
+      for (int tile = lo; tile < hi; ++tile, ++k) {
+        while (tile >= tile_pre[g + 1]) ++g;
+        if (g != cur_g) {
+          if (cur_g >= 0) mma_commit(&q_empty[qseq & 1]);
+          ++qseq;
+          if (!mbar_wait(&q_full[qseq & 1], (qseq >> 1) & 1, abort_flag)) break;
+          cur_g = g;
+        }
+        const int acc = k & 1;
+        if (!mbar_wait(&acc_empty[acc], ((k >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&full[stage], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(kbuf + stage * tile_bytes);
+        const uint32_t b0 = smem_u32(qbuf + (qseq & 1) * q_bytes);
+        const uint32_t d = tmem_base + (uint32_t)(acc * n_mma);
+        for (int kk = 0; kk < p.Di / 32; ++kk)
+          mma_e4m3(d, smem_desc_kmajor(a0 + kk * 32, p.Di), smem_desc_kmajor(b0 + kk * 32, p.Di),
+                   idesc, kk > 0 ? 1u : 0u);
+        mma_commit(&empty[stage]);
+        mma_commit(&acc_full[acc]);
+        if (++stage == p.stages) { stage = 0; ph ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue warpgroups
+    const int wg = (warp - 2) >> 2;
+    const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int m = quad * 32 + lane;
+    int g = g_first, k = 0;
+    for (int tile = lo; tile < hi; ++tile, ++k) {
+      while (tile >= tile_pre[g + 1]) ++g;
+      if ((k & 1) != wg) continue;
+      const int acc = k & 1;
+      if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const int b = g / p.groups_per_b;
+      const int t0 = (g % p.groups_per_b) * p.nq;
+      const int j = (tile - tile_pre[g]) * kTileM + m;
+      for (int qi = 0; qi < p.nq; ++qi) {
+        const int t = t0 + qi;
+        if (t >= p.Tq) break;                   // warp-uniform
+        const size_t row = (size_t)b * p.Tq + t;
+        const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * p.Hi);
+        float s = 0.0f;
+        for (int h0 = 0; h0 < p.Hi; h0 += 32) {
+          float v[32];
+          tmem_ld_32(tmem_base + ((uint32_t)(quad * 32) << 16) +
+                         (uint32_t)(acc * n_mma + qi * p.Hi + h0), v);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 wv = __ldg(w4 + (h0 + i) / 4);
+            s = fmaf(wv.x, fmaxf(v[i], 0.0f), s);
+            s = fmaf(wv.y, fmaxf(v[i + 1], 0.0f), s);
+            s = fmaf(wv.z, fmaxf(v[i + 2], 0.0f), s);
+            s = fmaf(wv.w, fmaxf(v[i + 3], 0.0f), s);
+          }
+        }
+        if (j < min(p.nvalid[row], p.N)) p.scores[row * p.N + j] = s;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.ncols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) record_error(p.err, CSA2_ERR_TIMEOUT);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* ptr, uint64_t rows, int row_bytes, int box_rows) {
+  auto encode = get_encode();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
+                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+
+bool index_score_tc_supported(int B, int Tq, int Hi, int Di, const int32_t* cand) {
+  if (cand != nullptr) return false;
+  if (!(Di == 64 || Di == 128)) return false;
+  if (!(Hi == 64 || Hi == 128)) return false;
+  const int nq = Tq == 1 ? 1 : min(Tq, 256 / Hi);
+  const long long G = (long long)B * ((Tq + nq - 1) / nq);
+  return G >= 1 && G <= kMaxGroups;
+}
+
+cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
+                                  int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
+                                  float* scores, int* err, cudaStream_t stream) {
+  TcParams p;
+  p.Tq = Tq;
+  p.N = N;
+  p.Hi = Hi;
+  p.Di = Di;
+  p.nq = Tq == 1 ? 1 : min(Tq, 256 / Hi);
+  p.groups_per_b = (Tq + p.nq - 1) / p.nq;
+  p.G = B * p.groups_per_b;
+  const int n_mma = Hi * p.nq;
+  p.ncols = 32;
+  while (p.ncols < (uint32_t)(2 * n_mma)) p.ncols <<= 1;
+  p.stages = n_mma <= 64 ? 8 : 5;
+  p.nvalid = nvalid;
+  p.idx_w = idx_w;
+  p.scores = scores;
+  p.err = err;
+
+  CUtensorMap kmap, qmap;
+  if (!make_map(&kmap, idx_k, (uint64_t)B * N, Di, kTileM) ||
+      !make_map(&qmap, idx_q, (uint64_t)B * Tq * Hi, Di, n_mma))
+    return cudaErrorInvalidValue;
+
+  const size_t smem = 1024 + (size_t)p.stages * kTileM * Di + 2 * (size_t)n_mma * Di +
+                      (2 * p.stages + 8) * sizeof(uint64_t) + 16 + (p.G + 1 + 32) * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  // upper bound on the tile count; CTAs beyond the real count get empty ranges
+  const long long max_tiles = (long long)p.G * ((N + kTileM - 1) / kTileM);
+  const int grid = (int)std::min<long long>(sm_count(), std::max<long long>(1, max_tiles));
+  index_score_tc_kernel<<<grid, kThreads, smem, stream>>>(kmap, qmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2
