@@ -9,10 +9,13 @@
 // ascending order, padded with -1.
 //
 // One CTA per (b, t) row. Scores become order-preserving 32-bit keys (key 0 is
-// reserved for "not a candidate"), an MSB-first 8-bit radix select finds the
-// K-th key T and how many entries equal to T are still needed, and an ordered
-// compaction writes every entry above T plus the first needed entries equal to
-// T, in id order. Rows that fit are staged once in shared memory.
+// reserved for "not a candidate"). The row's key range [kmin, kmax] is cut into
+// 4096 equal power-of-two bins (so the histogram adapts to where the scores
+// actually lie), a suffix scan finds the bin holding the K-th key, and the few
+// keys of that bin are ranked exactly against each other. A crowded threshold
+// bin (many equal scores) falls back to an MSB-first 8-bit radix select. The
+// selection is written in id order by a two-pass, ballot-based compaction.
+// Rows that fit are staged once in shared memory.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,12 +24,21 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSmemKeyCap = 48 * 1024;   // 192 KB of staged keys
+constexpr int kBins = 4096;
+constexpr int kBinsPerThread = kBins / kThreads;
+constexpr int kCandCap = 512;            // exact in-bin ranking up to this many keys
+constexpr int kSmemKeyCap = 40 * 1024;   // 160 KB of staged keys
 
 struct Scratch {
   uint32_t hist[256];
   int warp_sum[kWarps];
   int bcast[4];
+  int bins[kBins];
+  uint32_t cand_key[kCandCap];
+  int cand_pos[kCandCap];
+  int wgt[kWarps], weq[kWarps];
+  uint32_t red_min[kWarps], red_max[kWarps];
+  int ncand;
 };
 
 // Exclusive prefix sum over the block; returns this thread's prefix and the
@@ -112,37 +124,151 @@ __device__ void radix_select(const Row& r, int k, uint32_t& T, int& need_eq, Scr
 }
 
 // Writes, in ascending id order, every entry with key > T plus the first
-// `need_eq` entries with key == T, then pads with -1 up to `k`.
+// `need_eq` entries with key == T (T = 0 selects every real entry), then pads
+// with -1 up to `k`. Warp w owns a contiguous segment of the row; pass 1 counts,
+// pass 2 writes with ballot prefix counts.
 __device__ void ordered_emit(const Row& r, uint32_t T, int need_eq, int k, int32_t* out,
                              Scratch& sc, int* err) {
-  const int per = ceil_div(r.n, kThreads);
-  const int i0 = min(r.n, threadIdx.x * per), i1 = min(r.n, i0 + per);
-  int n_eq = 0;
-  for (int i = i0; i < i1; ++i) n_eq += key_at(r, i, err) == T ? 1 : 0;
-  int tot;
-  const int eq_before = block_exclusive_scan(n_eq, tot, sc);
-  int n_sel = 0, eq_seen = eq_before;
-  for (int i = i0; i < i1; ++i) {
-    uint32_t key = key_at(r, i, err);
-    if (key > T) ++n_sel;
-    else if (key == T && key != 0u && eq_seen++ < need_eq) ++n_sel;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = ceil_div(ceil_div(r.n, kWarps), 32) * 32;
+  const int w0 = min(r.n, warp * seg), w1 = min(r.n, w0 + seg);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int cnt_gt = 0, cnt_eq = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < w1 ? key_at(r, i, err) : 0u;
+    cnt_gt += __popc(__ballot_sync(0xffffffffu, key > T));
+    cnt_eq += __popc(__ballot_sync(0xffffffffu, key == T && key != 0u));
   }
-  int written;
-  int pos = block_exclusive_scan(n_sel, written, sc);
-  eq_seen = eq_before;
-  for (int i = i0; i < i1; ++i) {
-    uint32_t key = key_at(r, i, err);
-    bool take = key > T || (key == T && key != 0u && eq_seen++ < need_eq);
-    if (take) out[pos++] = r.cand ? r.cand[i] : i;
+  if (lane == 0) {
+    sc.wgt[warp] = cnt_gt;
+    sc.weq[warp] = cnt_eq;
   }
-  for (int i = written + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+  __syncthreads();
+  int eq_before = 0, pos = 0, total = 0;
+  {
+    int eqb = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int sel = sc.wgt[w] + min(sc.weq[w], max(0, need_eq - eqb));
+      if (w < warp) {
+        pos += sel;
+        eq_before += sc.weq[w];
+      }
+      total += sel;
+      eqb += sc.weq[w];
+    }
+  }
+  int eq_seen = eq_before;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < w1 ? key_at(r, i, err) : 0u;
+    const bool eq = key == T && key != 0u;
+    const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+    const bool take = key > T || (eq && eq_seen + __popc(eqmask & lt_mask) < need_eq);
+    const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tmask & lt_mask)] = r.cand ? r.cand[i] : i;
+    pos += __popc(tmask);
+    eq_seen += __popc(eqmask);
+  }
+  for (int i = total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+  __syncthreads();
 }
 
-__device__ void select_into(const Row& r, int n_valid, int k, int32_t* out, Scratch& sc,
-                            int* err) {
+struct Range {
+  uint32_t kmin;
+  int shift;
+};
+
+__device__ __forceinline__ int bin_of(uint32_t key, Range rg) {
+  return (int)((key - rg.kmin) >> rg.shift);
+}
+
+// Histogram of the real keys over kBins bins of the row's key range.
+__device__ void build_hist(const Row& r, Range rg, Scratch& sc, int* err) {
+  for (int i = threadIdx.x; i < kBins; i += kThreads) sc.bins[i] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < r.n; i += kThreads) {
+    const uint32_t key = key_at(r, i, err);
+    if (key != 0u) atomicAdd(&sc.bins[bin_of(key, rg)], 1);
+  }
+  __syncthreads();
+}
+
+// Finds (T, need_eq) for the k-th largest real key, 1 <= k <= n_valid.
+__device__ void find_threshold(const Row& r, Range rg, int k, uint32_t& T, int& need_eq,
+                               Scratch& sc, int* err) {
+  // bins in descending order: thread t owns bins kBins-1-4t .. kBins-4-4t
+  int local[kBinsPerThread];
+  int mine = 0;
+#pragma unroll
+  for (int j = 0; j < kBinsPerThread; ++j) {
+    local[j] = sc.bins[kBins - 1 - kBinsPerThread * threadIdx.x - j];
+    mine += local[j];
+  }
+  int tot;
+  int above = block_exclusive_scan(mine, tot, sc);
+  if (above < k && k <= above + mine) {
+#pragma unroll
+    for (int j = 0; j < kBinsPerThread; ++j) {
+      if (above < k && k <= above + local[j]) {
+        sc.bcast[0] = kBins - 1 - kBinsPerThread * (int)threadIdx.x - j;
+        sc.bcast[1] = k - above;   // how many to take from the bin
+        sc.bcast[2] = local[j];
+      }
+      above += local[j];
+    }
+  }
+  if (threadIdx.x == 0) sc.ncand = 0;
+  __syncthreads();
+  const int bT = sc.bcast[0], rT = sc.bcast[1], cT = sc.bcast[2];
+  if (cT > kCandCap) {
+    // crowded bin: exact radix select over the whole row
+    radix_select(r, k, T, need_eq, sc, err);
+    return;
+  }
+  for (int i = threadIdx.x; i < r.n; i += kThreads) {
+    const uint32_t key = key_at(r, i, err);
+    if (key != 0u && bin_of(key, rg) == bT) {
+      const int slot = atomicAdd(&sc.ncand, 1);
+      if (slot < kCandCap) {
+        sc.cand_key[slot] = key;
+        sc.cand_pos[slot] = i;
+      }
+    }
+  }
+  __syncthreads();
+  const int c = min(sc.ncand, kCandCap);
+  for (int s = threadIdx.x; s < c; s += kThreads) {
+    const uint32_t ks = sc.cand_key[s];
+    const int ps = sc.cand_pos[s];
+    int gt = 0, eqb = 0;
+    for (int u = 0; u < c; ++u) {
+      const uint32_t ku = sc.cand_key[u];
+      gt += ku > ks;
+      eqb += (ku == ks) && (sc.cand_pos[u] < ps);
+    }
+    if (gt + eqb == rT - 1) {
+      sc.bcast[0] = (int)ks;
+      sc.bcast[1] = eqb + 1;
+    }
+  }
+  __syncthreads();
+  T = (uint32_t)sc.bcast[0];
+  need_eq = sc.bcast[1];
+  __syncthreads();
+}
+
+__device__ void select_into(const Row& r, int n_valid, Range rg, bool& hist_ready, int k,
+                            int32_t* out, Scratch& sc, int* err) {
   uint32_t T = 0;
   int need_eq = 0;
-  if (n_valid > k) radix_select(r, k, T, need_eq, sc, err);
+  if (n_valid > k) {
+    if (!hist_ready) {
+      build_hist(r, rg, sc, err);
+      hist_ready = true;
+    }
+    find_threshold(r, rg, k, T, need_eq, sc, err);
+  }
   ordered_emit(r, T, need_eq, k, out, sc, err);
 }
 
@@ -154,35 +280,62 @@ topk_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict_
   extern __shared__ uint32_t staged[];
   __shared__ Scratch sc;
   const size_t row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Row r;
   r.s = scores + row * ld;
   r.cand = cand ? cand + row * ld : nullptr;
   r.keys = nullptr;
   r.n = cand ? ld : max(0, min(ld, nvalid[row]));
 
-  // count the real candidates (and stage their keys); check the pool's order
+  // stage the keys; count the real ones and find their range; check the pool's order
   int mine = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
   bool nan = false, unsorted = false;
   for (int i = threadIdx.x; i < r.n; i += kThreads) {
     uint32_t key;
     if (r.cand) {
-      int32_t id = r.cand[i];
+      const int32_t id = r.cand[i];
       if (i > 0 && id >= 0 && (r.cand[i - 1] < 0 || r.cand[i - 1] >= id)) unsorted = true;
       key = id < 0 ? 0u : rank_key(r.s[i], nan);
     } else {
       key = rank_key(r.s[i], nan);
     }
     if (kStage) staged[i] = key;
-    mine += key != 0u;
+    if (key != 0u) {
+      ++mine;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
   }
   if (nan) record_error(err, CSA2_ERR_NONFINITE);
   if (unsorted) record_error(err, CSA2_ERR_DEVICE_INDEX);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sc.red_min[warp] = kmin;
+    sc.red_max[warp] = kmax;
+  }
   int n_valid;
   block_exclusive_scan(mine, n_valid, sc);   // also a barrier for the staged keys
   if (kStage) r.keys = staged;
+  Range rg;
+  kmin = sc.red_min[0];
+  kmax = sc.red_max[0];
+  for (int w = 1; w < kWarps; ++w) {
+    kmin = min(kmin, sc.red_min[w]);
+    kmax = max(kmax, sc.red_max[w]);
+  }
+  rg.kmin = kmin;
+  const uint32_t span = kmax >= kmin ? kmax - kmin : 0u;   // largest offset
+  const int bits = span == 0u ? 0 : 32 - __clz(span);      // offsets fit in `bits` bits
+  rg.shift = bits > 12 ? bits - 12 : 0;                    // -> at most 4096 bins
+  bool hist_ready = false;
 
-  select_into(r, n_valid, K, topk_out + row * K, sc, err);
-  if (cand_out) select_into(r, n_valid, Cout, cand_out + row * Cout, sc, err);
+  select_into(r, n_valid, rg, hist_ready, K, topk_out + row * K, sc, err);
+  if (cand_out) select_into(r, n_valid, rg, hist_ready, Cout, cand_out + row * Cout, sc, err);
 }
 
 }  // namespace

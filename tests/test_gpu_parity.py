@@ -119,12 +119,18 @@ def _scores(rng, shape, kind):
         return x
     if kind == "wide":
         return (rng.standard_normal(shape) * 1e4).astype(np.float32)
+    if kind == "const":
+        return np.full(shape, 7.0, np.float32)
+    if kind == "twovals":
+        return np.where(rng.random(shape) < 0.5, 3.0, -2.0).astype(np.float32)
+    if kind == "gauss_int":       # like the indexer scores: integers ~ N(4800, 1000)
+        return np.round(rng.normal(4800, 1000, shape)).astype(np.float32)
     raise ValueError(kind)
 
 
 @pytest.mark.parametrize("ld,K", [(3000, 64), (3000, 1), (4096, 256), (32768, 2048), (70000, 2048),
                                   (100, 200)])
-@pytest.mark.parametrize("kind", ["ties", "signed", "wide"])
+@pytest.mark.parametrize("kind", ["ties", "signed", "wide", "const", "twovals", "gauss_int"])
 def test_topk_bit_exact(ld, K, kind):
     rng = np.random.default_rng(ld + K)
     rows = 6
