@@ -36,4 +36,12 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
                                float* lse, void* workspace, int* err, cudaStream_t stream);
 
+// Tensor-core attention kernel (attn_tc.cu); partials go to ws_o/ws_ml when nsplit > 1.
+int sparse_attn_tc_max_split_len();
+cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
+                                  const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
+                                  int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
+                                  int nsplit, int split_len, uint16_t* out, float* lse,
+                                  float* ws_o, float2* ws_ml, int* err, cudaStream_t stream);
+
 }  // namespace csa2

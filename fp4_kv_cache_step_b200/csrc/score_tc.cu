@@ -39,7 +39,7 @@ constexpr int kThreads = 320;
 constexpr int kMaxGroups = 8192;
 
 struct TcParams {
-  int Tq, N, Hi, Di, nq, G, groups_per_b, stages;
+  int Tq, N, Hi, Di, nq, G, groups_per_b, stages, nacc;
   uint32_t ncols;
   const int32_t* nvalid;
   const float* idx_w;
@@ -70,8 +70,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   uint64_t* full = reinterpret_cast<uint64_t*>(qbuf + 2 * q_bytes);
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* q_full = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + 4;
+  uint64_t* q_full = acc_empty + 4;
   uint64_t* q_empty = q_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -113,9 +113,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
@@ -186,8 +188,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           if (!mbar_wait(&q_full[qseq & 1], (qseq >> 1) & 1, abort_flag)) break;
           cur_g = g;
         }
-        const int acc = k & 1;
-        if (!mbar_wait(&acc_empty[acc], ((k >> 1) & 1) ^ 1, abort_flag)) break;
+        const int acc = k % p.nacc;
+        if (!mbar_wait(&acc_empty[acc], ((k / p.nacc) & 1) ^ 1, abort_flag)) break;
         if (!mbar_wait(&full[stage], ph, abort_flag)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(kbuf + stage * tile_bytes);
@@ -206,28 +208,61 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
     const int m = quad * 32 + lane;
-    int g = g_first, k = 0;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    int g = g_first, k = 0, wg_group = -1;
+    float wreg[64];                            // head weights of the current query (nq == 1)
+    int nv_cur = 0;
     for (int tile = lo; tile < hi; ++tile, ++k) {
       while (tile >= tile_pre[g + 1]) ++g;
       if ((k & 1) != wg) continue;
-      const int acc = k & 1;
-      if (!mbar_wait(&acc_full[acc], (k >> 1) & 1, abort_flag)) break;
-      tc_fence_after();
+      const int acc = k % p.nacc;
       const int b = g / p.groups_per_b;
       const int t0 = (g % p.groups_per_b) * p.nq;
+      if (p.nq == 1 && p.Hi == 64 && g != wg_group) {
+        // load this query's weights and length once per group, before the wait
+        const size_t row = (size_t)b * p.Tq + t0;
+        const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 wv = __ldg(w4 + i);
+          wreg[4 * i] = wv.x;
+          wreg[4 * i + 1] = wv.y;
+          wreg[4 * i + 2] = wv.z;
+          wreg[4 * i + 3] = wv.w;
+        }
+        nv_cur = min(__ldg(p.nvalid + row), p.N);
+        wg_group = g;
+      }
+      if (!mbar_wait_warp(&acc_full[acc], (k / p.nacc) & 1, abort_flag)) break;
+      tc_fence_after();
       const int j = (tile - tile_pre[g]) * kTileM + m;
+      const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(acc * n_mma);
+      if (p.nq == 1 && p.Hi == 64) {
+        float v[64];
+        tmem_ld_64(acc_addr, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          s0 = fmaf(wreg[i], fmaxf(v[i], 0.0f), s0);
+          s1 = fmaf(wreg[i + 1], fmaxf(v[i + 1], 0.0f), s1);
+        }
+        if (j < nv_cur) p.scores[((size_t)b * p.Tq + t0) * p.N + j] = s0 + s1;
+        continue;
+      }
       for (int qi = 0; qi < p.nq; ++qi) {
         const int t = t0 + qi;
         if (t >= p.Tq) break;                   // warp-uniform
         const size_t row = (size_t)b * p.Tq + t;
         const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * p.Hi);
         float s = 0.0f;
-        for (int h0 = 0; h0 < p.Hi; h0 += 32) {
-          float v[32];
-          tmem_ld_32(tmem_base + ((uint32_t)(quad * 32) << 16) +
-                         (uint32_t)(acc * n_mma + qi * p.Hi + h0), v);
+        for (int h0 = 0; h0 < p.Hi; h0 += 64) {
+          float v[64];
+          tmem_ld_64(acc_addr + (uint32_t)(qi * p.Hi + h0), v);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
+          for (int i = 0; i < 64; i += 4) {
             const float4 wv = __ldg(w4 + (h0 + i) / 4);
             s = fmaf(wv.x, fmaxf(v[i], 0.0f), s);
             s = fmaf(wv.y, fmaxf(v[i + 1], 0.0f), s);
@@ -310,8 +345,9 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
   p.groups_per_b = (Tq + p.nq - 1) / p.nq;
   p.G = B * p.groups_per_b;
   const int n_mma = Hi * p.nq;
+  p.nacc = n_mma <= 128 ? 4 : 2;          // accumulator ring depth
   p.ncols = 32;
-  while (p.ncols < (uint32_t)(2 * n_mma)) p.ncols <<= 1;
+  while (p.ncols < (uint32_t)(p.nacc * n_mma)) p.ncols <<= 1;
   p.stages = n_mma <= 64 ? 8 : 5;
   p.nvalid = nvalid;
   p.idx_w = idx_w;
@@ -324,7 +360,7 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
     return cudaErrorInvalidValue;
 
   const size_t smem = 1024 + (size_t)p.stages * kTileM * Di + 2 * (size_t)n_mma * Di +
-                      (2 * p.stages + 8) * sizeof(uint64_t) + 16 + (p.G + 1 + 32) * sizeof(int);
+                      (2 * p.stages + 12) * sizeof(uint64_t) + 16 + (p.G + 1 + 32) * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -78,13 +78,34 @@ struct Row {
   int n;                // entries in the row
 };
 
-__device__ __forceinline__ uint32_t key_at(const Row& r, int i, int* err) {
-  if (r.keys) return r.keys[i];
-  if (r.cand && r.cand[i] < 0) return 0u;
+constexpr int kBatch = 8;   // independent loads in flight per thread
+
+// Keys at positions base + stride * j (j < kBatch); 0 past `end`.
+__device__ __forceinline__ void keys_batch(const Row& r, int base, int stride, int end,
+                                           uint32_t (&k)[kBatch], int* err) {
+  if (r.keys) {
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + stride * j;
+      k[j] = i < end ? r.keys[i] : 0u;
+    }
+    return;
+  }
+  float f[kBatch];
+  int32_t c[kBatch];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    const int i = base + stride * j;
+    f[j] = i < end ? __ldg(r.s + i) : 0.0f;
+    c[j] = (r.cand && i < end) ? __ldg(r.cand + i) : 0;
+  }
   bool nan = false;
-  uint32_t k = rank_key(r.s[i], nan);
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    const int i = base + stride * j;
+    k[j] = (i < end && c[j] >= 0) ? rank_key(f[j], nan) : 0u;
+  }
   if (nan) record_error(err, CSA2_ERR_NONFINITE);
-  return k;
 }
 
 // Finds the key T of the k-th largest non-zero key (1 <= k <= number of
@@ -96,14 +117,21 @@ __device__ void radix_select(const Row& r, int k, uint32_t& T, int& need_eq, Scr
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256; i += kThreads) sc.hist[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < r.n; i += kThreads) {
-      uint32_t key = key_at(r, i, err);
-      bool match = key != 0u && (key & mask) == prefix;
-      uint32_t digit = (key >> shift) & 0xffu;
-      // aggregate equal digits within the warp before touching shared memory
-      uint32_t peers = __match_any_sync(__activemask(), match ? digit : 0x100u);
-      if (match && (__ffs(peers) - 1) == (threadIdx.x & 31))
-        atomicAdd(&sc.hist[digit], (uint32_t)__popc(peers));
+    // the loop bound is warp-uniform so every lane reaches __match_any_sync
+    const int lane = threadIdx.x & 31;
+    for (int w0 = threadIdx.x - lane; w0 < r.n; w0 += kThreads * kBatch) {
+      uint32_t kb[kBatch];
+      keys_batch(r, w0 + lane, kThreads, r.n, kb, err);
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const uint32_t key = kb[j];
+        const bool match = key != 0u && (key & mask) == prefix;
+        const uint32_t digit = (key >> shift) & 0xffu;
+        // aggregate equal digits within the warp before touching shared memory
+        const uint32_t peers = __match_any_sync(0xffffffffu, match ? digit : 0x100u);
+        if (match && (__ffs(peers) - 1) == (threadIdx.x & 31))
+          atomicAdd(&sc.hist[digit], (uint32_t)__popc(peers));
+      }
     }
     __syncthreads();
     int v = threadIdx.x < 256 ? (int)sc.hist[255 - threadIdx.x] : 0;
@@ -134,11 +162,14 @@ __device__ void ordered_emit(const Row& r, uint32_t T, int need_eq, int k, int32
   const int w0 = min(r.n, warp * seg), w1 = min(r.n, w0 + seg);
   const uint32_t lt_mask = (1u << lane) - 1u;
   int cnt_gt = 0, cnt_eq = 0;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < w1 ? key_at(r, i, err) : 0u;
-    cnt_gt += __popc(__ballot_sync(0xffffffffu, key > T));
-    cnt_eq += __popc(__ballot_sync(0xffffffffu, key == T && key != 0u));
+  for (int base = w0; base < w1; base += 32 * kBatch) {
+    uint32_t kb[kBatch];
+    keys_batch(r, base + lane, 32, w1, kb, err);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      cnt_gt += __popc(__ballot_sync(0xffffffffu, kb[j] > T));
+      cnt_eq += __popc(__ballot_sync(0xffffffffu, kb[j] == T && kb[j] != 0u));
+    }
   }
   if (lane == 0) {
     sc.wgt[warp] = cnt_gt;
@@ -159,16 +190,21 @@ __device__ void ordered_emit(const Row& r, uint32_t T, int need_eq, int k, int32
     }
   }
   int eq_seen = eq_before;
-  for (int base = w0; base < w1; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < w1 ? key_at(r, i, err) : 0u;
-    const bool eq = key == T && key != 0u;
-    const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
-    const bool take = key > T || (eq && eq_seen + __popc(eqmask & lt_mask) < need_eq);
-    const uint32_t tmask = __ballot_sync(0xffffffffu, take);
-    if (take) out[pos + __popc(tmask & lt_mask)] = r.cand ? r.cand[i] : i;
-    pos += __popc(tmask);
-    eq_seen += __popc(eqmask);
+  for (int base = w0; base < w1; base += 32 * kBatch) {
+    uint32_t kb[kBatch];
+    keys_batch(r, base + lane, 32, w1, kb, err);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = base + lane + 32 * j;
+      const uint32_t key = kb[j];
+      const bool eq = key == T && key != 0u;
+      const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+      const bool take = key > T || (eq && eq_seen + __popc(eqmask & lt_mask) < need_eq);
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(tmask & lt_mask)] = r.cand ? r.cand[i] : i;
+      pos += __popc(tmask);
+      eq_seen += __popc(eqmask);
+    }
   }
   for (int i = total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
   __syncthreads();
@@ -187,9 +223,12 @@ __device__ __forceinline__ int bin_of(uint32_t key, Range rg) {
 __device__ void build_hist(const Row& r, Range rg, Scratch& sc, int* err) {
   for (int i = threadIdx.x; i < kBins; i += kThreads) sc.bins[i] = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < r.n; i += kThreads) {
-    const uint32_t key = key_at(r, i, err);
-    if (key != 0u) atomicAdd(&sc.bins[bin_of(key, rg)], 1);
+  for (int i0 = threadIdx.x; i0 < r.n; i0 += kThreads * kBatch) {
+    uint32_t kb[kBatch];
+    keys_batch(r, i0, kThreads, r.n, kb, err);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      if (kb[j] != 0u) atomicAdd(&sc.bins[bin_of(kb[j], rg)], 1);
   }
   __syncthreads();
 }
@@ -226,13 +265,17 @@ __device__ void find_threshold(const Row& r, Range rg, int k, uint32_t& T, int& 
     radix_select(r, k, T, need_eq, sc, err);
     return;
   }
-  for (int i = threadIdx.x; i < r.n; i += kThreads) {
-    const uint32_t key = key_at(r, i, err);
-    if (key != 0u && bin_of(key, rg) == bT) {
-      const int slot = atomicAdd(&sc.ncand, 1);
-      if (slot < kCandCap) {
-        sc.cand_key[slot] = key;
-        sc.cand_pos[slot] = i;
+  for (int i0 = threadIdx.x; i0 < r.n; i0 += kThreads * kBatch) {
+    uint32_t kb[kBatch];
+    keys_batch(r, i0, kThreads, r.n, kb, err);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (kb[j] != 0u && bin_of(kb[j], rg) == bT) {
+        const int slot = atomicAdd(&sc.ncand, 1);
+        if (slot < kCandCap) {
+          sc.cand_key[slot] = kb[j];
+          sc.cand_pos[slot] = i0 + kThreads * j;
+        }
       }
     }
   }
@@ -290,24 +333,26 @@ topk_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict_
   // stage the keys; count the real ones and find their range; check the pool's order
   int mine = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  bool nan = false, unsorted = false;
-  for (int i = threadIdx.x; i < r.n; i += kThreads) {
-    uint32_t key;
-    if (r.cand) {
-      const int32_t id = r.cand[i];
-      if (i > 0 && id >= 0 && (r.cand[i - 1] < 0 || r.cand[i - 1] >= id)) unsorted = true;
-      key = id < 0 ? 0u : rank_key(r.s[i], nan);
-    } else {
-      key = rank_key(r.s[i], nan);
-    }
-    if (kStage) staged[i] = key;
-    if (key != 0u) {
-      ++mine;
-      kmin = min(kmin, key);
-      kmax = max(kmax, key);
+  bool unsorted = false;
+  for (int i0 = threadIdx.x; i0 < r.n; i0 += kThreads * kBatch) {
+    uint32_t kb[kBatch];
+    keys_batch(r, i0, kThreads, r.n, kb, err);
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = i0 + kThreads * j;
+      if (i >= r.n) break;
+      if (r.cand && i > 0) {
+        const int32_t id = __ldg(r.cand + i), prev = __ldg(r.cand + i - 1);
+        if (id >= 0 && (prev < 0 || prev >= id)) unsorted = true;
+      }
+      if (kStage) staged[i] = kb[j];
+      if (kb[j] != 0u) {
+        ++mine;
+        kmin = min(kmin, kb[j]);
+        kmax = max(kmax, kb[j]);
+      }
     }
   }
-  if (nan) record_error(err, CSA2_ERR_NONFINITE);
   if (unsorted) record_error(err, CSA2_ERR_DEVICE_INDEX);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {

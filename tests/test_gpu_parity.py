@@ -195,15 +195,34 @@ def _attn_case(seed, B, Tq, Hq, N, K, pad_frac=0.1, max_valid=None):
 @pytest.mark.parametrize("B,Tq,Hq,N,K", [(2, 1, 64, 4096, 256), (1, 1, 16, 4096, 256),
                                          (1, 2, 128, 2048, 200), (3, 1, 64, 16384, 2048),
                                          (40, 1, 64, 4096, 100), (1, 3, 48, 1024, 64)])
-@pytest.mark.parametrize("scale", [1.0 / math.sqrt(512.0), 1.0])
+@pytest.mark.parametrize("scale", [1.0 / math.sqrt(512.0), 1.0, 24.0])
 def test_sparse_attn_within_tolerance(B, Tq, Hq, N, K, scale):
     packed, sc, q, idx = _attn_case(B * 7 + K, B, Tq, Hq, N, K)
     idx[0, 0, :] = -1                                   # a row with nothing selected
     want, want_lse = oracle.sparse_attn(q, packed, sc, idx, scale)
     out, lse = csa2.csa2_sparse_attn(bf16_dev(q), dev(packed), dev(sc), dev(idx), scale)
-    assert_attn_close(host(out), want, "out")
+    assert_attn_close(host(out), want, "out", sharp=scale > 4.0)
     assert_lse_close(host(lse), want_lse, "lse")
     assert np.all(host(out)[0, 0] == 0.0)
+
+
+def test_sparse_attn_rising_max_across_tiles():
+    """Logits that grow tile after tile force the running max to be raised and
+    the accumulated output to be rescaled many times."""
+    B, Tq, Hq, N, K = 2, 1, 64, 4096, 1024
+    packed, sc, q, idx = _attn_case(77, B, Tq, Hq, N, K, pad_frac=0.0)
+    V = oracle.fp4_kv_unpack(packed, sc)
+    qf = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    for b in range(B):
+        logits = qf[b, 0] @ V[b].T                     # [Hq][N]
+        order = np.argsort(logits[0])                  # head 0: ascending logit
+        idx[b, 0] = np.sort(order[-K:]).astype(np.int32)
+        idx[b, 0] = order[-K:].astype(np.int32)        # unsorted: rising logits along the list
+    for scale in (8.0, 40.0):
+        want, want_lse = oracle.sparse_attn(q, packed, sc, idx, scale)
+        out, lse = csa2.csa2_sparse_attn(bf16_dev(q), dev(packed), dev(sc), dev(idx), scale)
+        assert_attn_close(host(out), want, "out scale=%g" % scale, sharp=True)
+        assert_lse_close(host(lse), want_lse, "lse scale=%g" % scale)
 
 
 def test_sparse_attn_bad_index_is_flagged_and_skipped():
