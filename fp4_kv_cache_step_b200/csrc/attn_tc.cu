@@ -17,7 +17,8 @@
 //   O   += P(t) V(t)  M=64 heads, N=256 dims (two halves), K=256 entries:
 //                     32 MMAs per tile, accumulator in TMEM lanes 0-15, all 512
 //                     columns.
-// V is dequantised twice into a ring of 32 KB shared-memory stages: first as
+// V is dequantised (with integer ops; values carry an exact factor 2^-8 that the
+// softmax scale and the epilogue undo) twice into a ring of 32 KB stages: first as
 // 64-dim K atoms of all 256 entries (K-major B operand of S), then as 32-entry
 // slices of all 512 dims (MN-major B operand of P V). The softmax is exact in
 // two passes over the CTA's (at most 512) scores, so O is never rescaled.
@@ -38,7 +39,8 @@ constexpr int kD = kHeadDim;             // 512
 constexpr int kHB = 64;                  // heads per CTA
 constexpr int kT = 256;                  // entries per tile
 constexpr int kMaxTiles = 2;             // tiles per CTA
-constexpr int kStages = 3;               // shared-memory ring depth
+constexpr int kStages = 2;               // fp16 ring depth
+constexpr int kRawBytes = 6 * 4096;      // raw (packed + scale) bytes of one stage: 6 x 16 B per thread
 constexpr int kStageBytes = 32768;
 constexpr int kAtom = 8192;              // 64 rows x 128 B (one K atom of Q or P)
 constexpr int kProducerWarps = 8;
@@ -58,11 +60,12 @@ struct Smem {
   uint32_t tmem_slot;
   int abort_flag;
   int idx[kMaxTiles][kT];
+  uint32_t valid[kMaxTiles][kT / 32];   // bit i of word w: entry 32 w + i is selected
   float head_scale[kHB];
 };
 
 constexpr size_t kSmemBytes = 1024 + 8 * kAtom /*Q*/ + kStages * kStageBytes + 4 * kAtom /*P*/ +
-                              sizeof(Smem);
+                              2 * kRawBytes /*raw ring*/ + sizeof(Smem);
 
 // byte offset of 16-byte chunk c (0..7) of row r in a [rows][128 B] swizzled block
 __device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
@@ -99,12 +102,6 @@ __device__ __forceinline__ void producer_bar() {
   asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
-__device__ __forceinline__ void ldg_nc_v4(const void* p, uint4& v) {
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-}
-
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -131,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   uint8_t* qs = base;                              // [8 atoms][64 heads][128 B]
   uint8_t* ring = qs + 8 * kAtom;                  // kStages x 32 KB
   uint8_t* ps = ring + kStages * kStageBytes;      // [4 atoms][64 heads][128 B]
-  Smem& sm = *reinterpret_cast<Smem*>(ps + 4 * kAtom);
+  uint8_t* rawbuf = ps + 4 * kAtom;                // 2 x [6 fields][256 threads][16 B]
+  Smem& sm = *reinterpret_cast<Smem*>(rawbuf + 2 * kRawBytes);
   volatile int* abort_flag = &sm.abort_flag;
 
   const size_t row = blockIdx.x;
@@ -181,6 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         }
       }
       const int tid = threadIdx.x;   // 0..255: one entry of each tile
+      const uint8_t* pk_row0 = p.kv_packed + (size_t)b * p.N * (kD / 2);
+      const uint8_t* sc_row0 = p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
 #pragma unroll
       for (int t = 0; t < kMaxTiles; ++t) {
         const int kk = k_begin + t * kT + tid;
@@ -190,6 +190,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           id = -1;
         }
         sm.idx[t][tid] = id;
+        const uint32_t vb = __ballot_sync(0xffffffffu, id >= 0);
+        if (lane == 0) sm.valid[t][tid >> 5] = vb;
+        if (id >= 0) {
+          // the stages read every row in 32- to 64-byte pieces: bring the whole
+          // packed row (256 B) and scale row (512 B) into L2 once, now
+          const uint8_t* pr = pk_row0 + (size_t)id * (kD / 2);
+          const uint8_t* sr = sc_row0 + (size_t)(id / kBlockEntries) * kD;
+          asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(pr));
+          asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(pr + 128));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(sr + 128 * j));
+        }
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -223,7 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         *reinterpret_cast<uint4*>(dst + swz(hh, c0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(dst + swz(hh, c0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         const float down = __uint_as_float((uint32_t)(127 - e) << 23);
-        if (lane == 0) sm.head_scale[hh] = hh < nh ? p.softmax_scale * kLog2e * down : 0.0f;
+        // x 2^8: the dequantised keys/values carry a factor 2^-8
+        if (lane == 0) sm.head_scale[hh] = hh < nh ? p.softmax_scale * kLog2e * down * 256.0f : 0.0f;
       }
       fence_async_smem();
       producer_bar();                         // indices visible to every producer warp
@@ -232,91 +245,155 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     }
 
     // ------------------------------------------------------------ V stages
-    // Stage k < 8 nt: K atom (k % 8) of tile k / 8, thread = entry.
-    // Stage k >= 8 nt: 32-entry slice of a tile, warp = 64-dim atom, lane = entry.
-    // Each warp keeps the loads of the next two stages in flight.
+    // Stage k < 8 nt: K atom a = k % 8 of tile k / 8; four lanes per entry, each
+    //   16 channels, four passes of 64 entries (a warp instruction touches 8 rows).
+    // Stage k >= 8 nt: 32-entry slice of a tile; eight lanes per entry, one
+    //   64-channel atom each (a warp instruction reads 4 whole rows).
+    // Each thread keeps the loads of the next two stages in flight (6 x 16 B).
     const uint8_t* pk_b = p.kv_packed + (size_t)b * p.N * (kD / 2);
     const uint8_t* sc_b = p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
     const int nstages = 16 * nt;
-    auto stage_src = [&](int k, int& id, int& atom) {
-      if (k < 8 * nt) {
-        id = sm.idx[k >> 3][threadIdx.x];
-        atom = k & 7;
-      } else {
-        const int kk = k - 8 * nt;
-        id = sm.idx[kk >> 3][(kk & 7) * 32 + lane];
-        atom = warp;
-      }
+    const int tid = threadIdx.x;
+    // Raw bytes of stage k go to raw slot k & 1 with cp.async (completion tracked
+    // per thread by commit groups, so the gather of stage k + 2 stays in flight
+    // while stage k is dequantised). Field f of thread tid is at f * 4096 + tid * 16.
+    auto cp16 = [](uint8_t* dst, const uint8_t* src) {
+      asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                   : "memory");
     };
-    auto issue = [&](int k, uint4 (&raw)[6]) {
-      if (k >= nstages) return;
-      int id, atom;
-      stage_src(k, id, atom);
-      if (id >= 0) {
-        const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + atom * 32;
-        const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + atom * 64;
-        // volatile: issued here, two stages before their use, not sunk to it
-        ldg_nc_v4(pr, raw[0]);
-        ldg_nc_v4(pr + 16, raw[1]);
-        ldg_nc_v4(sr, raw[2]);
-        ldg_nc_v4(sr + 16, raw[3]);
-        ldg_nc_v4(sr + 32, raw[4]);
-        ldg_nc_v4(sr + 48, raw[5]);
-      }
+    auto cp8 = [](uint8_t* dst, const uint8_t* src) {
+      asm volatile("cp.async.ca.shared.global.L2::256B [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src)
+                   : "memory");
     };
-    // one stage: wait for its slot, dequantise the registers loaded two stages
-    // ago, refill them with stage k + 2, store, publish
-    auto run_stage = [&](int k, uint4 (&cur)[6]) -> bool {
-      const int st = k % kStages;
-      if (!mbar_wait_warp(&sm.bar.empty[st], ((k / kStages) & 1) ^ 1, abort_flag)) return false;
-      int id, atom;
-      stage_src(k, id, atom);
-      uint4 v[8];
-      if (id >= 0) {
-        const uint32_t cw[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w,
-                                cur[1].x, cur[1].y, cur[1].z, cur[1].w};
-        const uint32_t sw[16] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y,
-                                 cur[3].z, cur[3].w, cur[4].x, cur[4].y, cur[4].z, cur[4].w,
-                                 cur[5].x, cur[5].y, cur[5].z, cur[5].w};
+    auto issue = [&](int k) {
+      if (k < nstages) {
+        uint8_t* raw = rawbuf + (k & 1) * kRawBytes + tid * 16;
+        if (k < 8 * nt) {
+          const int t = k >> 3, atom = k & 7, sub = tid & 3;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t h[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const __half2 vv = e2m1x2_to_half2((uint8_t)(cw[j] >> (8 * t)));
-            const __half2 ss = e4m3x2_to_half2((uint16_t)(sw[2 * j + (t >> 1)] >> (16 * (t & 1))));
-            const __half2 r = __hmul2(vv, ss);
-            h[t] = *reinterpret_cast<const uint32_t*>(&r);
+          for (int ps = 0; ps < 4; ++ps) {
+            const int id = sm.idx[t][ps * 64 + (tid >> 2)];
+            if (id >= 0) {
+              cp16(raw + ps * 4096, sc_b + (size_t)(id / kBlockEntries) * kD + atom * 64 + sub * 16);
+              cp8(raw + (4 + (ps >> 1)) * 4096 + (ps & 1) * 8,
+                  pk_b + (size_t)id * (kD / 2) + atom * 32 + sub * 8);
+            }
           }
-          v[j] = make_uint4(h[0], h[1], h[2], h[3]);
+        } else {
+          const int kk = k - 8 * nt;
+          const int id = sm.idx[kk >> 3][(kk & 7) * 32 + (tid >> 3)];
+          const int atom = tid & 7;
+          if (id >= 0) {
+            const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + atom * 32;
+            const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + atom * 64;
+            cp16(raw, pr);
+            cp16(raw + 4096, pr + 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cp16(raw + (2 + j) * 4096, sr + 16 * j);
+          }
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = make_uint4(0, 0, 0, 0);
       }
-      issue(k + 2, cur);
-      uint8_t* dst = ring + st * kStageBytes;
-      if (k < 8 * nt) {
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto fetch = [&](int k, uint4 (&cur)[6]) {
+      asm volatile("cp.async.wait_group 1;" ::: "memory");   // stage k landed (k + 1 may not have)
+      const uint8_t* raw = rawbuf + (k & 1) * kRawBytes + tid * 16;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + swz(threadIdx.x, c)) = v[c];
-      } else {
+      for (int f = 0; f < 6; ++f) cur[f] = *reinterpret_cast<const uint4*>(raw + f * 4096);
+    };
+    // 8 E2M1 codes (one 32-bit word) times their 8 E4M3 scales (two words) -> one
+    // 16-byte chunk of fp16 values, times 2^-8. Integer ops only (byte permutes,
+    // shifts, one logic op): the conversion pipe stays free for the softmax.
+    //  - E2M1 magnitude m -> high byte of fp16(m) from an 8-entry byte table
+    //    (0, 0.5, 1, 1.5, 2, 3, 4, 6 -> 00 38 3C 3E 40 42 44 46), sign spliced in;
+    //  - a non-negative E4M3 byte shifted left by 7 is the fp16 of its value * 2^-8
+    //    (exponent bias 7 -> 15, mantissa 3 -> 10 bits; subnormals line up too);
+    //  - the fp16 product is exact (<= 6 significant bits, >= 2^-18).
+    auto dq8 = [](uint32_t codes, uint32_t s_lo, uint32_t s_hi) -> uint4 {
+      const uint32_t mag = codes & 0x77777777u;
+      const uint32_t m_lo = __byte_perm(0x3E3C3800u, 0x46444240u, mag);         // codes 0-3
+      const uint32_t m_hi = __byte_perm(0x3E3C3800u, 0x46444240u, mag >> 16);   // codes 4-7
+      const uint32_t t = codes << 4;    // sign of each even code -> bit 7 of its byte
+      uint32_t h[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(dst + warp * 4096 + swz(lane, c)) = v[c];
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t mg = __byte_perm(j < 2 ? m_lo : m_hi, 0u, (j & 1) ? 0x3424u : 0x1404u);
+        const uint32_t sg = __byte_perm(t, codes, (uint32_t)((4 + j) * 0x1100 + j * 0x0011));
+        const uint32_t v = (mg & 0x7fff7fffu) | (sg & 0x80008000u);
+        const uint32_t sc = __byte_perm(j < 2 ? s_lo : s_hi, 0u, (j & 1) ? 0x4342u : 0x4140u) << 7;
+        const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&v),
+                                  *reinterpret_cast<const __half2*>(&sc));
+        h[j] = *reinterpret_cast<const uint32_t*>(&r);
       }
+      return make_uint4(h[0], h[1], h[2], h[3]);
+    };
+    auto publish = [&](int st) {
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.full[st]);
+    };
+    // Each stage: wait for its raw bytes and its fp16 slot, dequantise, start
+    // the gather of stage k + 2 into the raw slot just consumed, store, publish.
+    auto stage_s = [&](int k) -> bool {
+      const int st = k % kStages;
+      uint4 cur[6];
+      fetch(k, cur);
+      if (!mbar_wait_warp(&sm.bar.empty[st], ((k / kStages) & 1) ^ 1, abort_flag)) return false;
+      const int t = k >> 3, sub = tid & 3;
+      uint4 v[8];
+#pragma unroll
+      for (int ps = 0; ps < 4; ++ps) {
+        const uint32_t keep = sm.idx[t][ps * 64 + (tid >> 2)] >= 0 ? 0xffffffffu : 0u;
+        const uint4 s = cur[ps];
+        const uint32_t c0 = (ps & 1) ? cur[4 + (ps >> 1)].z : cur[4 + (ps >> 1)].x;
+        const uint32_t c1 = (ps & 1) ? cur[4 + (ps >> 1)].w : cur[4 + (ps >> 1)].y;
+        const uint4 d0 = dq8(c0, s.x, s.y), d1 = dq8(c1, s.z, s.w);   // branch-free
+        v[2 * ps] = make_uint4(d0.x & keep, d0.y & keep, d0.z & keep, d0.w & keep);
+        v[2 * ps + 1] = make_uint4(d1.x & keep, d1.y & keep, d1.z & keep, d1.w & keep);
+      }
+      issue(k + 2);   // after the raw slot's values were consumed
+      uint8_t* dst = ring + st * kStageBytes;
+#pragma unroll
+      for (int ps = 0; ps < 4; ++ps) {
+        const int e = ps * 64 + (tid >> 2);
+        *reinterpret_cast<uint4*>(dst + swz(e, 2 * sub)) = v[2 * ps];
+        *reinterpret_cast<uint4*>(dst + swz(e, 2 * sub + 1)) = v[2 * ps + 1];
+      }
+      publish(st);
       return true;
     };
-    // two statically addressed register sets (the stage count is even)
-    uint4 ra[6], rb[6];
-    issue(0, ra);
-    issue(1, rb);
-    for (int k = 0; k < nstages; k += 2) {
-      if (!run_stage(k, ra)) break;
-      if (!run_stage(k + 1, rb)) break;
-    }
+    auto stage_pv = [&](int k) -> bool {
+      const int st = k % kStages;
+      uint4 cur[6];
+      fetch(k, cur);
+      if (!mbar_wait_warp(&sm.bar.empty[st], ((k / kStages) & 1) ^ 1, abort_flag)) return false;
+      const int kk = k - 8 * nt;
+      const int e = tid >> 3, atom = tid & 7;
+      const uint32_t keep = sm.idx[kk >> 3][(kk & 7) * 32 + e] >= 0 ? 0xffffffffu : 0u;
+      uint4 v[8];
+      const uint32_t cw[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w,
+                              cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+      const uint32_t sw[16] = {cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y,
+                               cur[3].z, cur[3].w, cur[4].x, cur[4].y, cur[4].z, cur[4].w,
+                               cur[5].x, cur[5].y, cur[5].z, cur[5].w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 d = dq8(cw[j], sw[2 * j], sw[2 * j + 1]);   // branch-free
+        v[j] = make_uint4(d.x & keep, d.y & keep, d.z & keep, d.w & keep);
+      }
+      issue(k + 2);   // after the raw slot's values were consumed
+      uint8_t* dst = ring + st * kStageBytes + atom * 4096;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + swz(e, c)) = v[c];
+      publish(st);
+      return true;
+    };
+    issue(0);
+    issue(1);
+    bool go = true;
+    for (int k = 0; go && k < 8 * nt; ++k) go = stage_s(k);
+    for (int k = 8 * nt; go && k < nstages; ++k) go = stage_pv(k);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");   // nothing in flight at exit
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -382,9 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         for (int c0 = 0; c0 < kT; c0 += 64) {
           float s[64];
           tmem_ld_64(tmem + lane_addr + 256u * t + c0, s);
+          const uint32_t v0 = sm.valid[t][c0 / 32], v1 = sm.valid[t][c0 / 32 + 1];
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (sm.idx[t][c0 + c] >= 0) m = fmaxf(m, s[c] * hs);
+            m = fmaxf(m, (((c < 32 ? v0 : v1) >> (c & 31)) & 1u) ? s[c] * hs : -INFINITY);
         }
       }
     }
@@ -396,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       for (int c0 = 0; c0 < kT; c0 += 64) {
         float s[64];
         tmem_ld_64(tmem + lane_addr + 256u * t + c0, s);
+        const uint32_t vw0 = sm.valid[t][c0 / 32], vw1 = sm.valid[t][c0 / 32 + 1];
         uint8_t* dst = ps + (c0 / 64) * kAtom;
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -403,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int i0 = 8 * c + 2 * u;
-            const bool v0 = sm.idx[t][c0 + i0] >= 0, v1 = sm.idx[t][c0 + i0 + 1] >= 0;
+            const uint32_t vw = i0 < 32 ? vw0 : vw1;
+            const bool v0 = (vw >> (i0 & 31)) & 1u, v1 = (vw >> ((i0 + 1) & 31)) & 1u;
             const float p0 = (v0 && m != -INFINITY) ? exp2f(s[i0] * hs - m) : 0.0f;
             const float p1 = (v1 && m != -INFINITY) ? exp2f(s[i0 + 1] * hs - m) : 0.0f;
             l += p0 + p1;
@@ -426,7 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       tc_fence_after();
       const bool o_owner = lane < 16 && h < nh;
       const size_t slot = (row * p.nhb + hb) * p.nsplit + split;
-      const float inv = l_o > 0.0f ? 1.0f / l_o : 0.0f;
+      // x 2^8 undoes the 2^-8 carried by the dequantised values
+      const float inv = l_o > 0.0f ? 256.0f / l_o : 0.0f;
 #pragma unroll 1
       for (int c0 = 0; c0 < kD; c0 += 64) {
         float o[64];
@@ -447,7 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         } else {
           float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + c0);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          for (int c = 0; c < 16; ++c)
+            dst[c] = make_float4(256.0f * o[4 * c], 256.0f * o[4 * c + 1], 256.0f * o[4 * c + 2],
+                                 256.0f * o[4 * c + 3]);
         }
       }
       if (lane < 16 && h < nh) {

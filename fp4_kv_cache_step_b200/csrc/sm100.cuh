@@ -56,13 +56,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Waits until the phase of parity `parity` has completed. Returns false (and
 // raises *abort for the rest of the CTA) if the wait runs out or another role
-// already gave up. The abort flag and the clock are read only every 64 polls so
-// that spinning threads add little shared-memory traffic.
+// already gave up. After a few polls the waiting thread sleeps between polls,
+// and the abort flag and the clock are read only every 64 polls, so waiting
+// costs the CTA's working warps little issue bandwidth or shared-memory traffic.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    // back off so that waiting warps leave issue slots to the working ones
+    if (it > 8u) __nanosleep(it > 64u ? 256u : 32u);
     if ((it & 63u) == 0u) {
       if (*abort) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
