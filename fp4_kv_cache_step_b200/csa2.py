@@ -48,7 +48,7 @@ class LayerArgs(ctypes.Structure):
 EXPORTS = ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk",
            "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn",
            "csa2_layer_step_workspace_bytes", "csa2_layer_step", "csa2_check_device_errors",
-           "csa2_last_error")
+           "csa2_last_error", "csa2_sparse_attn_noalloc")
 
 _lib = None
 
@@ -70,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.csa2_sparse_attn_workspace_bytes.argtypes = [I, I, I, I, I]
     L.csa2_sparse_attn_workspace_bytes.restype = Z
     L.csa2_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
+    L.csa2_sparse_attn_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P]
     L.csa2_layer_step_workspace_bytes.argtypes = [ctypes.POINTER(LayerArgs), I,
                                                   ctypes.POINTER(SharedState)]
     L.csa2_layer_step_workspace_bytes.restype = Z
@@ -78,7 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.csa2_last_error.argtypes = []
     L.csa2_last_error.restype = ctypes.c_char_p
     for f in ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk", "csa2_sparse_attn",
-              "csa2_layer_step", "csa2_check_device_errors"):
+              "csa2_layer_step", "csa2_check_device_errors", "csa2_sparse_attn_noalloc"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -204,6 +205,29 @@ def csa2_sparse_attn(q: torch.Tensor, kv_packed: torch.Tensor, kv_scale: torch.T
                               float(softmax_scale), _p(out), _p(lse if want_lse else None),
                               _p(workspace) if need else None, need, _stream(q.device)),
            "csa2_sparse_attn")
+    return out, (lse if want_lse else None)
+
+
+def csa2_sparse_attn_noalloc(q: torch.Tensor, kv_packed: torch.Tensor, kv_scale: torch.Tensor,
+                             topk_idx: torch.Tensor, softmax_scale: float, want_lse: bool = True,
+                             out: Optional[torch.Tensor] = None,
+                             lse: Optional[torch.Tensor] = None):
+    """csa2_sparse_attn for callers that cannot allocate device memory: the
+    library's built-in scratch array stands in for the workspace (outputs are
+    still the caller's). Calls that overlap on the GPU must be avoided."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want(topk_idx, torch.int32, "topk_idx", 3)
+    B, Tq, Hq, D = q.shape
+    N = kv_packed.shape[1]
+    K = topk_idx.shape[-1]
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=q.device)
+    _check(load().csa2_sparse_attn_noalloc(_p(q), _p(kv_packed), _p(kv_scale), _p(topk_idx), B, Tq,
+                                           Hq, D, N, K, float(softmax_scale), _p(out),
+                                           _p(lse if want_lse else None), _stream(q.device)),
+           "csa2_sparse_attn_noalloc")
     return out, (lse if want_lse else None)
 
 

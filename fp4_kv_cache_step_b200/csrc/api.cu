@@ -132,6 +132,19 @@ size_t layer_scores_bytes(const csa2_layer_args* a, csa2_mode mode, const csa2_s
 
 }  // namespace
 
+// Internal helpers shared with the other exported entry points' files.
+namespace csa2 {
+csa2_status api_check_attn_args(const uint16_t* q, const uint8_t* kv_packed,
+                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
+                                int Hq, int D, int N, int K, const uint16_t* out, const float* lse) {
+  return check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
+}
+int* api_error_word(cudaError_t* e) { return device_error_word(e); }
+csa2_status api_fail(csa2_status s, const char* msg) { return fail(s, "%s", msg); }
+csa2_status api_cuda_fail(cudaError_t e, const char* where) { return cuda_fail(e, where); }
+csa2_status api_ok() { return ok(); }
+}  // namespace csa2
+
 extern "C" {
 
 csa2_status fp4_kv_pack(const float* kv, int B, int N, int D, uint8_t* kv_packed,

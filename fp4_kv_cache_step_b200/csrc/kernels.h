@@ -5,7 +5,19 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "csa2.h"
+
 namespace csa2 {
+
+// Argument checks, error word and last-error text of api.cu, for entry points
+// that live in other files.
+csa2_status api_check_attn_args(const uint16_t* q, const uint8_t* kv_packed,
+                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
+                                int Hq, int D, int N, int K, const uint16_t* out, const float* lse);
+int* api_error_word(cudaError_t* e);
+csa2_status api_fail(csa2_status s, const char* msg);
+csa2_status api_cuda_fail(cudaError_t e, const char* where);
+csa2_status api_ok();
 
 cudaError_t launch_fp4_pack(const float* kv, int B, int N, int D, uint8_t* packed,
                             uint8_t* scale, int* err, cudaStream_t stream);

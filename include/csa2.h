@@ -172,6 +172,35 @@ CSA2_API csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packe
                              void* workspace, size_t workspace_bytes, csa2_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_sparse_attn_noalloc -- csa2_sparse_attn without a caller workspace.
+ * (An interface addition of this library; the pages describe no such call.)
+ *
+ * For callers that cannot allocate device memory at all: code inside an engine
+ * that owns and pre-partitions all device memory, a custom-op hook that offers
+ * no allocator, or a latency-critical path that must avoid an allocation and
+ * its implicit synchronisation. Same arguments, semantics and results as
+ * csa2_sparse_attn minus the workspace: the split scratch comes from a fixed
+ * device array of CSA2_NOALLOC_SCRATCH_BYTES built into the library (resident
+ * on every device that called this function, until the process exits).
+ *  - Returns CSA2_ERR_WORKSPACE, launching nothing, when the shape needs more
+ *    split scratch than the array holds (compare with
+ *    csa2_sparse_attn_workspace_bytes()).
+ *  - All calls on a device share the array: calls that overlap on the GPU
+ *    (e.g. two streams at once) race. The array keeps the last call's contents;
+ *    nothing in it needs to start at zero.
+ *  - The first call on each device looks up the array's address on the host;
+ *    make that first call before any stream capture.
+ *  - Calls no cudaMalloc, cudaFree or allocating library routine.
+ * ------------------------------------------------------------------------ */
+#define CSA2_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* kv_packed,
+                                              const uint8_t* kv_scale, const int32_t* topk_idx,
+                                              int B, int Tq, int Hq, int D, int N, int K,
+                                              float softmax_scale, uint16_t* out, float* lse,
+                                              csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa2_layer_step -- one CSA2 layer in its static mode ([N] "The Three Modes
  * Full Reindex And Reuse"; [M] 3.3, 3.4). The shared state holds non-owning
  * device pointers that several layers pass to each other without copies: the
