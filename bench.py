@@ -46,6 +46,17 @@ def rank_workload(w, rank: int):
     return w if rank == 0 else w.replace(seed=w.seed + 1000 * rank)
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (every rank takes part; NCCL on GPUs, gloo on CPU)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -191,11 +202,7 @@ def run_ours(args):
         barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     csa2.check_device_errors()
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = max_total_ms / args.steps
     value = world * args.steps / (max_total_ms / 1e3)
 
