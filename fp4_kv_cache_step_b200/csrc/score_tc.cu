@@ -37,9 +37,11 @@ using namespace sm100;
 constexpr int kTileM = 128;
 constexpr int kThreads = 320;
 constexpr int kMaxGroups = 8192;
+constexpr size_t kSmemLimit = 227 * 1024;   // opt-in dynamic shared memory per CTA
 
 struct TcParams {
   int Tq, N, Hi, Di, nq, G, groups_per_b, stages, nacc;
+  int sub;            // 128-entry MMA blocks per pipeline tile (2 for decode, 1 for prefill)
   uint32_t ncols;
   const int32_t* nvalid;
   const float* idx_w;
@@ -53,7 +55,23 @@ __device__ __forceinline__ int group_tiles(const TcParams& p, int g) {
   int nmax = 0;
   for (int t = t0; t < min(t0 + p.nq, p.Tq); ++t)
     nmax = max(nmax, min(p.N, max(0, p.nvalid[(size_t)b * p.Tq + t])));
-  return (nmax + kTileM - 1) / kTileM;
+  const int rows = kTileM * p.sub;
+  return (nmax + rows - 1) / rows;
+}
+
+// The MMAs of one pipeline tile: SUB blocks of 128 entries x KSTEPS steps of
+// 32 key bytes. Descriptor start addresses advance by adding (bytes >> 4) to
+// the low field (shared-memory addresses stay below 2^18, so no carry).
+template <int SUB, int KSTEPS>
+__device__ __forceinline__ void issue_tile(uint32_t d0, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                           uint32_t n_mma) {
+#pragma unroll
+  for (int sb = 0; sb < SUB; ++sb)
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk)
+      mma_e4m3(d0 + (uint32_t)sb * n_mma,
+               ad + (uint64_t)((sb * kTileM * KSTEPS * 32 + kk * 32) >> 4),
+               bd + (uint64_t)((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -62,7 +80,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const int tile_bytes = kTileM * p.Di;
+  const int tile_rows = kTileM * p.sub;
+  const int tile_bytes = tile_rows * p.Di;
   const int n_mma = p.Hi * p.nq;
   const int q_bytes = n_mma * p.Di;
   uint8_t* kbuf = base;
@@ -169,7 +188,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         const int e = tile - tile_pre[g];
         if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&full[stage], tile_bytes);
-        tma_load_2d(&kmap, &full[stage], kbuf + stage * tile_bytes, 0, b * p.N + e * kTileM);
+        tma_load_2d(&kmap, &full[stage], kbuf + stage * tile_bytes, 0, b * p.N + e * tile_rows);
         if (++stage == p.stages) { stage = 0; ph ^= 1; }
       }
     }
@@ -177,30 +196,41 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_e4m3_f32(kTileM, n_mma);
-      int stage = 0;
-      uint32_t ph = 0;
-      int qseq = -1, cur_g = -1, g = g_first, k = 0;
-      for (int tile = lo; tile < hi; ++tile, ++k) {
-        while (tile >= tile_pre[g + 1]) ++g;
+      const int ksteps = p.Di / 32;
+      const uint32_t acc_cols = (uint32_t)(n_mma * p.sub);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, acc_ph = 1;
+      int qseq = -1, cur_g = -1, g = g_first;
+      int next_g_tile = tile_pre[g + 1];
+      uint32_t b0 = 0;
+      for (int tile = lo; tile < hi; ++tile) {
+        if (tile >= next_g_tile) {
+          while (tile >= tile_pre[g + 1]) ++g;
+          next_g_tile = tile_pre[g + 1];
+        }
         if (g != cur_g) {
           if (cur_g >= 0) mma_commit(&q_empty[qseq & 1]);
           ++qseq;
           if (!mbar_wait(&q_full[qseq & 1], (qseq >> 1) & 1, abort_flag)) break;
           cur_g = g;
+          b0 = smem_u32(qbuf + (qseq & 1) * q_bytes);
         }
-        const int acc = k % p.nacc;
-        if (!mbar_wait(&acc_empty[acc], ((k / p.nacc) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[acc], acc_ph, abort_flag)) break;
         if (!mbar_wait(&full[stage], ph, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(kbuf + stage * tile_bytes);
-        const uint32_t b0 = smem_u32(qbuf + (qseq & 1) * q_bytes);
-        const uint32_t d = tmem_base + (uint32_t)(acc * n_mma);
-        for (int kk = 0; kk < p.Di / 32; ++kk)
-          mma_e4m3(d, smem_desc_kmajor(a0 + kk * 32, p.Di), smem_desc_kmajor(b0 + kk * 32, p.Di),
-                   idesc, kk > 0 ? 1u : 0u);
+        const uint64_t ad = smem_desc_kmajor(smem_u32(kbuf + stage * tile_bytes), p.Di);
+        const uint64_t bd = smem_desc_kmajor(b0, p.Di);
+        const uint32_t d0 = tmem_base + (uint32_t)acc * acc_cols;
+        if (p.sub == 2 && ksteps == 4)
+          issue_tile<2, 4>(d0, ad, bd, idesc, (uint32_t)n_mma);
+        else if (ksteps == 4)
+          issue_tile<1, 4>(d0, ad, bd, idesc, (uint32_t)n_mma);
+        else
+          issue_tile<1, 2>(d0, ad, bd, idesc, (uint32_t)n_mma);
         mma_commit(&empty[stage]);
         mma_commit(&acc_full[acc]);
         if (++stage == p.stages) { stage = 0; ph ^= 1; }
+        if (++acc == p.nacc) { acc = 0; acc_ph ^= 1; }
       }
     }
   } else {
@@ -235,21 +265,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       if (!mbar_wait_warp(&acc_full[acc], (k / p.nacc) & 1, abort_flag)) break;
       tc_fence_after();
-      const int j = (tile - tile_pre[g]) * kTileM + m;
-      const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(acc * n_mma);
+      const int j = (tile - tile_pre[g]) * (kTileM * p.sub) + m;
+      const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(acc * n_mma * p.sub);
       if (p.nq == 1 && p.Hi == 64) {
-        float v[64];
-        tmem_ld_64(acc_addr, v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        float s0 = 0.0f, s1 = 0.0f;
+        float* dst = p.scores + ((size_t)b * p.Tq + t0) * p.N;
+        for (int sb = 0; sb < p.sub; ++sb) {
+          float v[64];
+          tmem_ld_64(acc_addr + (uint32_t)(sb * 64), v);
+          if (sb == p.sub - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          }
+          float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          s0 = fmaf(wreg[i], fmaxf(v[i], 0.0f), s0);
-          s1 = fmaf(wreg[i + 1], fmaxf(v[i + 1], 0.0f), s1);
+          for (int i = 0; i < 64; i += 2) {
+            s0 = fmaf(wreg[i], fmaxf(v[i], 0.0f), s0);
+            s1 = fmaf(wreg[i + 1], fmaxf(v[i + 1], 0.0f), s1);
+          }
+          if (j + sb * kTileM < nv_cur) dst[j + sb * kTileM] = s0 + s1;
         }
-        if (j < nv_cur) p.scores[((size_t)b * p.Tq + t0) * p.N + j] = s0 + s1;
         continue;
       }
       for (int qi = 0; qi < p.nq; ++qi) {
@@ -345,27 +380,37 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
   p.groups_per_b = (Tq + p.nq - 1) / p.nq;
   p.G = B * p.groups_per_b;
   const int n_mma = Hi * p.nq;
+  // Decode (64 query columns): 256-entry pipeline tiles (32 KB of keys, two
+  // M = 128 blocks), so the per-tile barrier round trips are spread over
+  // twice the bytes; prefill keeps 128-entry tiles for its wider accumulators.
+  p.sub = (n_mma <= 64 && Di == 128) ? 2 : 1;
   p.nacc = n_mma <= 128 ? 4 : 2;          // accumulator ring depth
   p.ncols = 32;
-  while (p.ncols < (uint32_t)(p.nacc * n_mma)) p.ncols <<= 1;
-  p.stages = n_mma <= 64 ? 8 : 5;
+  while (p.ncols < (uint32_t)(p.nacc * n_mma * p.sub)) p.ncols <<= 1;
+  // key-tile ring: as deep as the shared memory left after the query
+  // buffers, barriers and the group prefix allows (at most 6 or 8 stages)
+  const size_t fixed = 1024 + 2 * (size_t)n_mma * Di + (2 * 16 + 12) * sizeof(uint64_t) + 16 +
+                       (size_t)(p.G + 1 + 32) * sizeof(int);
+  const size_t tile_bytes = (size_t)kTileM * p.sub * Di;
+  const int max_stages = p.sub == 2 ? 6 : (n_mma <= 64 ? 8 : 5);
+  p.stages = (int)std::min<size_t>(max_stages, (kSmemLimit - fixed) / tile_bytes);
+  if (p.stages < 2) return cudaErrorInvalidValue;
   p.nvalid = nvalid;
   p.idx_w = idx_w;
   p.scores = scores;
   p.err = err;
 
   CUtensorMap kmap, qmap;
-  if (!make_map(&kmap, idx_k, (uint64_t)B * N, Di, kTileM) ||
+  if (!make_map(&kmap, idx_k, (uint64_t)B * N, Di, kTileM * p.sub) ||
       !make_map(&qmap, idx_q, (uint64_t)B * Tq * Hi, Di, n_mma))
     return cudaErrorInvalidValue;
 
-  const size_t smem = 1024 + (size_t)p.stages * kTileM * Di + 2 * (size_t)n_mma * Di +
-                      (2 * p.stages + 12) * sizeof(uint64_t) + 16 + (p.G + 1 + 32) * sizeof(int);
+  const size_t smem = fixed + (size_t)p.stages * tile_bytes;
   cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // upper bound on the tile count; CTAs beyond the real count get empty ranges
-  const long long max_tiles = (long long)p.G * ((N + kTileM - 1) / kTileM);
+  const long long max_tiles = (long long)p.G * ((N + kTileM * p.sub - 1) / (kTileM * p.sub));
   const int grid = (int)std::min<long long>(sm_count(), std::max<long long>(1, max_tiles));
   index_score_tc_kernel<<<grid, kThreads, smem, stream>>>(kmap, qmap, p);
   return cudaGetLastError();
