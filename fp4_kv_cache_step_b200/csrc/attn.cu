@@ -14,7 +14,6 @@ namespace csa2 {
 namespace {
 
 constexpr int kHB = 64;                 // heads per CTA
-constexpr int kTile = 64;               // selected entries per tile
 constexpr int kD = kHeadDim;            // 512
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -66,21 +65,19 @@ int sm_count() {
   return n;
 }
 
-// Each CTA takes at most sparse_attn_tc_max_split_len() entries (two 256-entry
-// tiles); when the batch has too few rows to fill the GPU the index list is cut
-// further, down to one tile per CTA.
+// A CTA walks its split of the index list in tiles of sparse_attn_tc_tile()
+// entries, so any split length works; the list is split only when the batch
+// has too few (row, head block) pairs to give every SM a CTA.
 SplitPlan plan_splits(int rows, int Hq, int K) {
   SplitPlan p;
   p.nhb = ceil_div(Hq, kHB);
+  const int tile = sparse_attn_tc_tile();
   const int ctas = rows * p.nhb;
   const int sms = sm_count();
-  const int max_len = sparse_attn_tc_max_split_len();
-  const int min_split = ceil_div(K, max_len);
-  const int max_split = ceil_div(K, max_len / 2);
   int nsplit = ctas >= sms ? 1 : sms / ctas;
-  if (nsplit > max_split) nsplit = max_split;
-  if (nsplit < min_split) nsplit = min_split;
-  p.split_len = ceil_div(ceil_div(K, nsplit), kTile) * kTile;
+  nsplit = min(nsplit, ceil_div(K, tile));
+  nsplit = max(nsplit, 1);
+  p.split_len = ceil_div(ceil_div(K, nsplit), tile) * tile;
   p.nsplit = ceil_div(K, p.split_len);
   return p;
 }

@@ -49,7 +49,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                float* lse, void* workspace, int* err, cudaStream_t stream);
 
 // Tensor-core attention kernel (attn_tc.cu); partials go to ws_o/ws_ml when nsplit > 1.
-int sparse_attn_tc_max_split_len();
+int sparse_attn_tc_tile();
 cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,

@@ -90,10 +90,12 @@ def test_workspace_is_checked_before_launch(lib):
     rc = lib.csa2_sparse_attn(a, a, a, a, 2, 1, 64, 512, 4096, 2048, ctypes.c_float(1.0), a, None,
                               None, 0, None)
     assert _status(rc) == "WORKSPACE"
-    # enough rows for one CTA each and at most 512 selected entries: no split
+    # enough rows to give every SM a CTA: no split, whatever K
     assert lib.csa2_sparse_attn_workspace_bytes(4096, 1, 64, 512, 512) == 0
-    # 2048 entries are split four ways: partial outputs plus (max, sum) per head
-    assert lib.csa2_sparse_attn_workspace_bytes(4096, 1, 64, 512, 2048) >= 4096 * 4 * 64 * 512 * 4
+    assert lib.csa2_sparse_attn_workspace_bytes(4096, 1, 64, 512, 2048) == 0
+    # 32 rows on 148 SMs: the 2048 entries are split four ways, partial outputs
+    # plus (max, sum) per head
+    assert lib.csa2_sparse_attn_workspace_bytes(32, 1, 64, 512, 2048) >= 32 * 4 * 64 * 512 * 4
 
 
 def test_layer_step_rejects_bad_mode_and_pool(lib):
