@@ -16,6 +16,8 @@
 // bin (many equal scores) falls back to an MSB-first 8-bit radix select. The
 // selection is written in id order by a two-pass, ballot-based compaction.
 // Rows that fit are staged once in shared memory.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -383,12 +385,312 @@ topk_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict_
   if (cand_out) select_into(r, n_valid, rg, hist_ready, Cout, cand_out + row * Cout, sc, err);
 }
 
+
+// ---------------------------------------------------------------------------
+// Cluster variant: when there are too few rows to give every SM a CTA, each
+// row is cut into `cs` contiguous slices, one per CTA of a thread-block
+// cluster. Every CTA stages its slice's keys in shared memory; the CTAs agree
+// on the threshold through histograms summed over distributed shared memory
+// (12-bit digits refined from the row's key range down to the exact key T),
+// then each writes its part of the ascending output at an offset given by the
+// counts of the CTAs before it. Same ranking and output as topk_kernel.
+namespace cg = cooperative_groups;
+
+constexpr int kCThreads = 1024;
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kCBins = 4096;                    // one 12-bit digit per pass
+constexpr int kCBinsPerThread = kCBins / kCThreads;
+static_assert(kCBinsPerThread == 4, "the cluster histogram is read as one uint4 per thread");
+
+struct __align__(16) ClusterShared {
+  uint32_t hist[kCBins];      // this CTA's histogram of the current pass (read by the cluster)
+  uint32_t kmin, kmax;        // this CTA's key range
+  int nvalid;                 // real keys in this CTA's slice
+  int gt, eq;                 // keys > T and == T in this slice (emit)
+  int warp_sum[kCWarps];
+  int bcast[4];
+};
+
+__device__ __forceinline__ int cblock_exclusive_scan(int v, int& total, ClusterShared& sc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sc.warp_sum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = sc.warp_sum[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    sc.warp_sum[lane] = wi - w;
+    if (lane == 31) sc.bcast[3] = wi;
+  }
+  __syncthreads();
+  const int res = sc.warp_sum[warp] + incl - v;
+  total = sc.bcast[3];
+  __syncthreads();
+  return res;
+}
+
+// (T, need_eq) of the k-th largest real key of the row (1 <= k <= n_valid):
+// T is the key, need_eq how many keys equal to T the selection takes.
+__device__ void cluster_threshold(cg::cluster_group& cl, const uint32_t* keys, int nloc,
+                                  uint32_t kmin, uint32_t kmax, int k, uint32_t& T, int& need_eq,
+                                  ClusterShared& sc) {
+  const int cs = (int)cl.num_blocks();
+  uint32_t lo = kmin;
+  const uint32_t span = kmax - kmin;
+  int bits = span == 0u ? 0 : 32 - __clz(span);   // offsets from lo fit in `bits` bits
+  int shift = bits > 12 ? bits - 12 : 0;
+  uint32_t width_m1 = span;                        // current range is [lo, lo + width_m1]
+  int krem = k;
+  const int lane = threadIdx.x & 31;
+  for (;;) {
+    for (int i = threadIdx.x; i < kCBins; i += kCThreads) sc.hist[i] = 0;
+    __syncthreads();
+    for (int w0 = threadIdx.x - lane; w0 < nloc; w0 += kCThreads) {
+      const int i = w0 + lane;
+      const uint32_t key = i < nloc ? keys[i] : 0u;
+      const bool in = key != 0u && key - lo <= width_m1 && key >= lo;
+      if (in) atomicAdd(&sc.hist[(key - lo) >> shift], 1u);
+    }
+    cl.sync();
+    // bins in descending order: thread t owns bins kCBins-1-4t .. kCBins-4-4t,
+    // read as one 16-byte vector from every CTA of the cluster (loads first)
+    const int vb = kCBins - kCBinsPerThread * (threadIdx.x + 1);   // lowest of the four
+    uint4 part[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < cs) part[r] = *reinterpret_cast<const uint4*>(cl.map_shared_rank(&sc.hist[vb], r));
+    int local[kCBinsPerThread] = {0, 0, 0, 0};
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < cs) {
+        local[0] += (int)part[r].w;   // bin vb + 3 first: descending order
+        local[1] += (int)part[r].z;
+        local[2] += (int)part[r].y;
+        local[3] += (int)part[r].x;
+      }
+    }
+    const int mine = local[0] + local[1] + local[2] + local[3];
+    int total;
+    int above = cblock_exclusive_scan(mine, total, sc);
+    if (above < krem && krem <= above + mine) {
+#pragma unroll
+      for (int j = 0; j < kCBinsPerThread; ++j) {
+        if (above < krem && krem <= above + local[j]) {
+          sc.bcast[0] = kCBins - 1 - kCBinsPerThread * (int)threadIdx.x - j;
+          sc.bcast[1] = krem - above;
+        }
+        above += local[j];
+      }
+    }
+    __syncthreads();
+    const uint32_t bstar = (uint32_t)sc.bcast[0];
+    krem = sc.bcast[1];
+    // every CTA has read the others' histograms before any clears its own
+    cl.sync();
+    lo += bstar << shift;
+    if (shift == 0) {
+      T = lo;
+      need_eq = krem;
+      return;
+    }
+    width_m1 = (1u << shift) - 1u;
+    shift = shift > 12 ? shift - 12 : 0;
+  }
+}
+
+__global__ void __launch_bounds__(kCThreads, 1)
+topk_cluster_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict__ nvalid,
+                    const int32_t* __restrict__ cand, int K, int32_t* __restrict__ topk_out,
+                    int Cout, int32_t* __restrict__ cand_out, int slice, int* err) {
+  extern __shared__ uint32_t keys[];
+  __shared__ ClusterShared sc;
+  cg::cluster_group cl = cg::this_cluster();
+  const int cs = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  const size_t row = blockIdx.x / cs;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* srow = scores + row * ld;
+  const int32_t* crow = cand ? cand + row * ld : nullptr;
+  const int n = cand ? ld : max(0, min(ld, nvalid[row]));
+  const int i0 = min(n, rank * slice), i1 = min(n, i0 + slice);
+  const int nloc = i1 - i0;
+
+  // stage this slice's keys (kBatch loads in flight per thread); count the real
+  // ones and find their range
+  int mine = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  bool nan = false, unsorted = false;
+  for (int b0 = threadIdx.x; b0 < nloc; b0 += kCThreads * kBatch) {
+    float f[kBatch];
+    int32_t id[kBatch], prev[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = b0 + kCThreads * j;
+      const int gi = i0 + i;
+      f[j] = i < nloc ? __ldg(srow + gi) : 0.0f;
+      id[j] = (crow && i < nloc) ? __ldg(crow + gi) : 0;
+      prev[j] = (crow && i < nloc && gi > 0) ? __ldg(crow + gi - 1) : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = b0 + kCThreads * j;
+      if (i >= nloc) break;
+      if (crow && id[j] >= 0 && i0 + i > 0 && (prev[j] < 0 || prev[j] >= id[j])) unsorted = true;
+      const uint32_t key = id[j] >= 0 ? rank_key(f[j], nan) : 0u;
+      keys[i] = key;
+      if (key != 0u) {
+        ++mine;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+      }
+    }
+  }
+  if (nan) record_error(err, CSA2_ERR_NONFINITE);
+  if (unsorted) record_error(err, CSA2_ERR_DEVICE_INDEX);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  }
+  if (lane == 0) sc.warp_sum[warp] = mine;
+  if (threadIdx.x == 0) {
+    sc.kmin = 0xffffffffu;
+    sc.kmax = 0u;
+  }
+  __syncthreads();
+  if (lane == 0) {
+    atomicMin(&sc.kmin, kmin);
+    atomicMax(&sc.kmax, kmax);
+  }
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < kCWarps; ++w) tot += sc.warp_sum[w];
+    sc.nvalid = tot;
+  }
+  cl.sync();
+  uint32_t gmin = 0xffffffffu, gmax = 0u;
+  int n_valid = 0;
+  for (int r = 0; r < cs; ++r) {
+    ClusterShared* o = cl.map_shared_rank(&sc, r);
+    gmin = min(gmin, o->kmin);
+    gmax = max(gmax, o->kmax);
+    n_valid += o->nvalid;
+  }
+
+  for (int pass = 0; pass < 2; ++pass) {
+    const int k = pass == 0 ? K : Cout;
+    int32_t* out = pass == 0 ? topk_out + row * (size_t)K : cand_out + row * (size_t)Cout;
+    if (pass == 1 && cand_out == nullptr) break;
+    uint32_t T = 0u;
+    int need_eq = 0;
+    if (n_valid > k) cluster_threshold(cl, keys, nloc, gmin, gmax, k, T, need_eq, sc);
+    // warp w takes a contiguous segment of the slice, its lanes interleaved
+    const int seg = ceil_div(ceil_div(nloc, kCWarps), 32) * 32;
+    const int w0 = min(nloc, warp * seg), w1 = min(nloc, w0 + seg);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int cnt_gt = 0, cnt_eq = 0;
+    for (int base = w0; base < w1; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < w1 ? keys[i] : 0u;
+      cnt_gt += __popc(__ballot_sync(0xffffffffu, key > T));
+      cnt_eq += __popc(__ballot_sync(0xffffffffu, key == T && key != 0u));
+    }
+    int tot_gt, tot_eq;
+    int gt_before_w = cblock_exclusive_scan(lane == 0 ? cnt_gt : 0, tot_gt, sc);
+    int eq_before_w = cblock_exclusive_scan(lane == 0 ? cnt_eq : 0, tot_eq, sc);
+    gt_before_w = __shfl_sync(0xffffffffu, gt_before_w, 0);
+    eq_before_w = __shfl_sync(0xffffffffu, eq_before_w, 0);
+    if (threadIdx.x == 0) {
+      sc.gt = tot_gt;
+      sc.eq = tot_eq;
+    }
+    cl.sync();
+    int gt_before = 0, eq_before = 0;
+    for (int r = 0; r < rank; ++r) {
+      ClusterShared* o = cl.map_shared_rank(&sc, r);
+      gt_before += o->gt;
+      eq_before += o->eq;
+    }
+    // entries selected before this warp: all > T keys of earlier CTAs and
+    // warps, and the first need_eq of the == T keys in order
+    int eq_seen = eq_before + eq_before_w;
+    int pos = gt_before + gt_before_w + min(eq_seen, need_eq);
+    for (int base = w0; base < w1; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < w1 ? keys[i] : 0u;
+      const bool eq = key == T && key != 0u;
+      const uint32_t eqmask = __ballot_sync(0xffffffffu, eq);
+      const bool take = key > T || (eq && eq_seen + __popc(eqmask & lt_mask) < need_eq);
+      const uint32_t tmask = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const int gi = i0 + i;
+        out[pos + __popc(tmask & lt_mask)] = crow ? crow[gi] : gi;
+      }
+      pos += __popc(tmask);
+      eq_seen += __popc(eqmask);
+    }
+    // padding: the last CTA of the cluster writes the -1 tail
+    if (rank == cs - 1) {
+      const int total = min(k, n_valid);
+      for (int i = total + threadIdx.x; i < k; i += kCThreads) out[i] = -1;
+    }
+    // the counts are read remotely before the next pass overwrites them
+    cl.sync();
+  }
+}
+
 }  // namespace
+
+int topk_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
 
 cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, const int32_t* cand,
                         int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
                         int* err, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
+  // Few rows: a cluster of cs CTAs per row (cs = 2, 4 or 8, as many as keep
+  // rows x cs within one wave), each staging a slice of the row.
+  const int sms = topk_sm_count();
+  int cs = 1;
+  while (cs < 8 && rows * cs * 2 <= sms) cs *= 2;
+  const size_t kSmemCap = 200 * 1024;
+  while (cs > 1 && cs < 8 && (size_t)ceil_div(ld, cs) * sizeof(uint32_t) > kSmemCap) cs *= 2;
+  const int slice = ceil_div(ld, cs);
+  if (cs > 1 && (size_t)slice * sizeof(uint32_t) <= kSmemCap) {
+    const size_t smem = (size_t)slice * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * cs), 1, 1);
+    cfg.blockDim = dim3(kCThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, nvalid, cand, K, topk_idx,
+                              Cout, cand_out, slice, err);
+  }
   if (ld <= kSmemKeyCap) {
     size_t smem = (size_t)ld * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>,
