@@ -311,11 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         mma_commit(&sm.bar.s_full[buf]);
         return true;
       };
-      if (ok && nt > 0) ok = issue_s(0);
-      if (ok && nt > 1) ok = issue_s(1);
-      for (int t = 0; ok && t < nt; ++t) {
+      auto issue_pv = [&](int t) {
         const int buf = t & 1;
-        if (!mbar_wait(&sm.bar.p_full[buf], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -326,7 +323,33 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
                     (t > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&sm.bar.v_free[buf]);
         mma_commit(&sm.bar.p_free[buf]);
-        if (t + 2 < nt) ok = issue_s(t + 2);
+      };
+      if (ok && nt > 0) ok = issue_s(0);
+      if (ok && nt > 1) ok = issue_s(1);
+      // Then whichever is ready first: P(t) V(t) once the softmax published P(t),
+      // or S(t') (t' <= t + 1: its S and P buffers were released by P(t'-2) V(t'-2))
+      // once the producers published its tile. Polling is bounded like mbar_wait.
+      int next_pv = 0, next_s = 2;
+      const uint64_t t0 = global_ns();
+      uint32_t spins = 0;
+      while (ok && next_pv < nt) {
+        bool did = false;
+        if (mbar_test_wait(&sm.bar.p_full[next_pv & 1], (next_pv >> 1) & 1)) {
+          issue_pv(next_pv++);
+          did = true;
+        }
+        if (next_s < nt && next_s <= next_pv + 1 &&
+            mbar_test_wait(&sm.bar.v_full[next_s & 1], (next_s >> 1) & 1)) {
+          ok = issue_s(next_s++);
+          did = true;
+        }
+        if (!did && (++spins & 63u) == 0u) {
+          __nanosleep(32);
+          if (*abort_flag || global_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            ok = false;
+          }
+        }
       }
       mma_commit(&sm.bar.o_full);
       // nothing may be in flight when TMEM is released
@@ -410,23 +433,47 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       if (!ok) break;
       tc_fence_after();
       const uint32_t vw0 = sm.valid[buf][0], vw1 = sm.valid[buf][1];
+      const bool all_valid = (vw0 & vw1) == 0xffffffffu;     // the same for every lane
       float y[64];
       tmem_ld_64(tmem + lane_addr + 64u * buf, y);
-      // logits in the log2 domain; the tile maximum over the selected entries
-      float ymax = -INFINITY;
+      // logits in the log2 domain relative to the current reference maximum,
+      // and their maximum over the selected entries
+      float xmax = -INFINITY;
+      if (all_valid) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        y[j] *= hs;
-        const bool v = (((j < 32 ? vw0 : vw1) >> (j & 31)) & 1u) != 0u;
-        ymax = fmaxf(ymax, v ? y[j] : -INFINITY);
+        for (int j = 0; j < 64; ++j) {
+          y[j] = fmaf(y[j], hs, -m_ref);
+          xmax = fmaxf(xmax, y[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          y[j] = fmaf(y[j], hs, -m_ref);
+          const bool v = (((j < 32 ? vw0 : vw1) >> (j & 31)) & 1u) != 0u;
+          xmax = fmaxf(xmax, v ? y[j] : -INFINITY);
+        }
       }
-      // lazy reference maximum: raise it only when P would exceed 2^8
+      // lazy reference maximum: raise it only when P would exceed 2^8 (always on
+      // the first tile with a selected entry, where the reference is -inf)
+      const bool raise = s_owner && xmax > kRescaleSlack;
       float alpha = 1.0f;
       const float m_old = m_ref;
-      if (s_owner && ymax > m_ref + kRescaleSlack) {
-        alpha = m_ref == -INFINITY ? 0.0f : exp2f(m_ref - ymax);
-        m_ref = ymax;
-        l *= alpha;
+      if (__any_sync(0xffffffffu, raise)) {
+        tmem_ld_64(tmem + lane_addr + 64u * buf, y);
+        float ymax = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          y[j] *= hs;
+          const bool v = (((j < 32 ? vw0 : vw1) >> (j & 31)) & 1u) != 0u;
+          ymax = fmaxf(ymax, v ? y[j] : -INFINITY);
+        }
+        if (raise) {
+          alpha = m_ref == -INFINITY ? 0.0f : exp2f(m_ref - ymax);
+          m_ref = ymax;
+          l *= alpha;
+        }
+#pragma unroll
+        for (int j = 0; j < 64; ++j) y[j] -= m_ref;
       }
       // O (lanes 0-15) is rescaled by its S lane's factor once P(t-1) V(t-1) is done
       const bool need = s_owner && alpha != 1.0f && m_old != -INFINITY;
@@ -450,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           tmem_st_32(tmem + lane_addr + c0, o);
         }
       }
-      // P = 2^(y - m_ref) in fp16 as the A operand of P V, and the row sum
+      // P = 2^y in fp16 (y <= 8) as the A operand of P V, and the row sum
       const bool live = s_owner && m_ref != -INFINITY;
       uint8_t* prow = ps + buf * kAtom;
 #pragma unroll
@@ -460,9 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         for (int u = 0; u < 4; ++u) {
           const int j = 8 * c + 2 * u;
           const uint32_t vw = j < 32 ? vw0 : vw1;
-          const bool v0 = live && ((vw >> (j & 31)) & 1u), v1 = live && ((vw >> ((j + 1) & 31)) & 1u);
-          const float p0 = v0 ? exp2f(y[j] - m_ref) : 0.0f;
-          const float p1 = v1 ? exp2f(y[j + 1] - m_ref) : 0.0f;
+          const bool v0 = live && (all_valid || ((vw >> (j & 31)) & 1u));
+          const bool v1 = live && (all_valid || ((vw >> ((j + 1) & 31)) & 1u));
+          const float p0 = v0 ? exp2f(y[j]) : 0.0f;
+          const float p1 = v1 ? exp2f(y[j + 1]) : 0.0f;
           l += p0 + p1;
           pk[u] = pack_half2(p0, p1);
         }
