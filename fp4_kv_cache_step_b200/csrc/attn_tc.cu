@@ -96,8 +96,31 @@ __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint
       : "memory");
 }
 
+// Same, with each descriptor given as its low word (start address and leading
+// offset: advancing it by (bytes >> 4) cannot carry out, shared-memory
+// addresses being below 2^18) and a common high word.
+__device__ __forceinline__ void mma_f16_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi_a,
+                                           uint32_t hi_b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %3};\n\t"
+      "mov.b64 db, {%2, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d),
+      "r"(a_lo), "r"(b_lo), "r"(hi_a), "r"(hi_b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 2^x with the hardware approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, far below the fp16 the probabilities are stored in)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -301,26 +324,34 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         if (!mbar_wait(&sm.bar.v_full[buf], (t >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t d = tmem + (16u << 16) + 64u * buf;
+        const uint32_t q_lo = (uint32_t)qd, q_hi = (uint32_t)(qd >> 32);
+        const uint32_t v_lo = (uint32_t)vk + (uint32_t)((buf * kVTile) >> 4);
+        const uint32_t v_hi = (uint32_t)(vk >> 32);
 #pragma unroll
         for (int a = 0; a < 8; ++a)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(d, qd + (uint64_t)((a * kAtom + kk * 32) >> 4),
-                    vk + (uint64_t)((buf * kVTile + a * kAtom + kk * 32) >> 4), id_s,
-                    (a > 0 || kk > 0) ? 1u : 0u);
+            mma_f16_lo(d, q_lo + (uint32_t)((a * kAtom + kk * 32) >> 4),
+                       v_lo + (uint32_t)((a * kAtom + kk * 32) >> 4), q_hi, v_hi, id_s,
+                       (a > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar.s_full[buf]);
         return true;
       };
       auto issue_pv = [&](int t) {
         const int buf = t & 1;
         tc_fence_after();
+        const uint32_t p_lo = (uint32_t)pd + (uint32_t)((buf * kAtom) >> 4);
+        const uint32_t p_hi = (uint32_t)(pd >> 32);
+        const uint32_t n_lo = (uint32_t)vn + (uint32_t)((buf * kVTile) >> 4);
+        const uint32_t n_hi = (uint32_t)(vn >> 32);
+        const uint32_t acc0 = t > 0 ? 1u : 0u;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int ks = 0; ks < kT / 16; ++ks)
-            mma_f16(tmem + 256u * h, pd + (uint64_t)((buf * kAtom + ks * 32) >> 4),
-                    vn + (uint64_t)((buf * kVTile + h * 4 * kAtom + ks * 2048) >> 4), id_o,
-                    (t > 0 || ks > 0) ? 1u : 0u);
+            mma_f16_lo(tmem + 256u * h, p_lo + (uint32_t)((ks * 32) >> 4),
+                       n_lo + (uint32_t)((h * 4 * kAtom + ks * 2048) >> 4), p_hi, n_hi, id_o,
+                       ks > 0 ? 1u : acc0);
         mma_commit(&sm.bar.v_free[buf]);
         mma_commit(&sm.bar.p_free[buf]);
       };
@@ -509,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           const uint32_t vw = j < 32 ? vw0 : vw1;
           const bool v0 = live && (all_valid || ((vw >> (j & 31)) & 1u));
           const bool v1 = live && (all_valid || ((vw >> ((j + 1) & 31)) & 1u));
-          const float p0 = v0 ? exp2f(y[j]) : 0.0f;
-          const float p1 = v1 ? exp2f(y[j + 1]) : 0.0f;
+          const float p0 = v0 ? fast_exp2(y[j]) : 0.0f;
+          const float p1 = v1 ? fast_exp2(y[j + 1]) : 0.0f;
           l += p0 + p1;
           pk[u] = pack_half2(p0, p1);
         }
