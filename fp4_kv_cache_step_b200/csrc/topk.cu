@@ -402,8 +402,15 @@ constexpr int kCBins = 4096;                    // one 12-bit digit per pass
 constexpr int kCBinsPerThread = kCBins / kCThreads;
 static_assert(kCBinsPerThread == 4, "the cluster histogram is read as one uint4 per thread");
 
+constexpr int kCCandCap = 512;                  // exact ranking of a threshold bin up to this size
+
 struct __align__(16) ClusterShared {
   uint32_t hist[kCBins];      // this CTA's histogram of the current pass (read by the cluster)
+  uint32_t cand_key[kCCandCap];   // this CTA's keys in the threshold bin (read by the cluster)
+  int cand_pos[kCCandCap];        // and their positions in the row
+  uint32_t all_key[kCCandCap];    // the threshold bin of the whole row
+  int all_pos[kCCandCap];
+  int ncand;
   uint32_t kmin, kmax;        // this CTA's key range
   int nvalid;                 // real keys in this CTA's slice
   int gt, eq;                 // keys > T and == T in this slice (emit)
@@ -441,7 +448,7 @@ __device__ __forceinline__ int cblock_exclusive_scan(int v, int& total, ClusterS
 
 // (T, need_eq) of the k-th largest real key of the row (1 <= k <= n_valid):
 // T is the key, need_eq how many keys equal to T the selection takes.
-__device__ void cluster_threshold(cg::cluster_group& cl, const uint32_t* keys, int nloc,
+__device__ void cluster_threshold(cg::cluster_group& cl, const uint32_t* keys, int nloc, int i0,
                                   uint32_t kmin, uint32_t kmax, int k, uint32_t& T, int& need_eq,
                                   ClusterShared& sc) {
   const int cs = (int)cl.num_blocks();
@@ -488,21 +495,76 @@ __device__ void cluster_threshold(cg::cluster_group& cl, const uint32_t* keys, i
         if (above < krem && krem <= above + local[j]) {
           sc.bcast[0] = kCBins - 1 - kCBinsPerThread * (int)threadIdx.x - j;
           sc.bcast[1] = krem - above;
+          sc.bcast[2] = local[j];
         }
         above += local[j];
       }
     }
+    if (threadIdx.x == 0) sc.ncand = 0;
     __syncthreads();
     const uint32_t bstar = (uint32_t)sc.bcast[0];
     krem = sc.bcast[1];
-    // every CTA has read the others' histograms before any clears its own
-    cl.sync();
+    const int cbin = sc.bcast[2];
     lo += bstar << shift;
     if (shift == 0) {
+      // every CTA has read the others' histograms before any clears its own
+      cl.sync();
       T = lo;
       need_eq = krem;
       return;
     }
+    if (cbin <= kCCandCap) {
+      // few keys in the threshold bin: gather them from the whole cluster and
+      // rank them exactly against each other (score desc, position asc)
+      const uint32_t bw_m1 = (1u << shift) - 1u;
+      for (int i = threadIdx.x; i < nloc; i += kCThreads) {
+        const uint32_t key = keys[i];
+        if (key != 0u && key >= lo && key - lo <= bw_m1) {
+          const int slot = atomicAdd(&sc.ncand, 1);
+          if (slot < kCCandCap) {
+            sc.cand_key[slot] = key;
+            sc.cand_pos[slot] = i0 + i;
+          }
+        }
+      }
+      cl.sync();   // candidate lists complete (and the histograms read)
+      int off = 0, c = 0;
+      for (int r = 0; r < cs; ++r) {
+        ClusterShared* o = cl.map_shared_rank(&sc, r);
+        const int nr = min(o->ncand, kCCandCap);
+        for (int u = threadIdx.x; u < nr; u += kCThreads) {
+          if (off + u < kCCandCap) {
+            sc.all_key[off + u] = o->cand_key[u];
+            sc.all_pos[off + u] = o->cand_pos[u];
+          }
+        }
+        off += nr;
+      }
+      c = min(off, kCCandCap);
+      __syncthreads();
+      for (int u = threadIdx.x; u < c; u += kCThreads) {
+        const uint32_t ku = sc.all_key[u];
+        const int pu = sc.all_pos[u];
+        int gt = 0, eqb = 0;
+        for (int v = 0; v < c; ++v) {
+          const uint32_t kv = sc.all_key[v];
+          gt += kv > ku;
+          eqb += (kv == ku) && (sc.all_pos[v] < pu);
+        }
+        if (gt + eqb == krem - 1) {
+          sc.bcast[0] = (int)ku;
+          sc.bcast[1] = eqb + 1;
+        }
+      }
+      __syncthreads();
+      T = (uint32_t)sc.bcast[0];
+      need_eq = sc.bcast[1];
+      // the candidate lists are read remotely: no CTA may rewrite its own
+      // before all have gathered (the caller's next cluster barrier)
+      return;
+    }
+    // every CTA has read the others' histograms before any clears its own
+    cl.sync();
     width_m1 = (1u << shift) - 1u;
     shift = shift > 12 ? shift - 12 : 0;
   }
@@ -594,7 +656,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int ld, const int32_t* __r
     if (pass == 1 && cand_out == nullptr) break;
     uint32_t T = 0u;
     int need_eq = 0;
-    if (n_valid > k) cluster_threshold(cl, keys, nloc, gmin, gmax, k, T, need_eq, sc);
+    if (n_valid > k) cluster_threshold(cl, keys, nloc, i0, gmin, gmax, k, T, need_eq, sc);
     // warp w takes a contiguous segment of the slice, its lanes interleaved
     const int seg = ceil_div(ceil_div(nloc, kCWarps), 32) * 32;
     const int w0 = min(nloc, warp * seg), w1 = min(nloc, w0 + seg);
