@@ -106,10 +106,11 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
     ws_o = static_cast<float*>(workspace);
     ws_ml = reinterpret_cast<float2*>(ws_o + slots * kHB * kD);
   }
+  bool merged = false;
   cudaError_t e = launch_sparse_attn_tc(q, kv_packed, kv_scale, topk_idx, rows, Tq, Hq, N, K,
                                         softmax_scale, p.nhb, p.nsplit, p.split_len, out, lse,
-                                        ws_o, ws_ml, err, stream);
-  if (e != cudaSuccess || p.nsplit == 1) return e;
+                                        ws_o, ws_ml, err, stream, &merged);
+  if (e != cudaSuccess || p.nsplit == 1 || merged) return e;
   attn_combine_kernel<<<dim3(rows, Hq), 128, 0, stream>>>(ws_o, ws_ml, Hq, p.nhb, p.nsplit, out,
                                                           lse);
   return cudaGetLastError();

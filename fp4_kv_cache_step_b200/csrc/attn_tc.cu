@@ -31,12 +31,16 @@
 // warps 9-12 stage Q, run the softmax (S rows in lanes 16-31 of their
 // quadrant), the O rescales and the epilogue (O rows in lanes 0-15). Every
 // mbarrier wait is bounded.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace csa2 {
 namespace {
+
+namespace cg = cooperative_groups;
 
 using namespace sm100;
 
@@ -64,6 +68,7 @@ struct Smem {
   int abort_flag;
   uint32_t valid[2][kT / 32];   // bit i of word w: entry 32 w + i of the tile is selected
   float head_scale[kHB];
+  float2 ml[kHB];               // this split's (reference maximum, row sum) per head
 };
 
 constexpr size_t kSmemBytes = 1024 + 8 * kAtom /*Q*/ + 2 * kVTile /*V*/ + 2 * kAtom /*P*/ +
@@ -166,7 +171,13 @@ struct AttnParams {
   float* ws_o;
   float2* ws_ml;
   int* err;
+  int cluster_merge;   // the splits of a (row, head block) form a cluster and merge in DSMEM
 };
+
+// float4 chunk c (0..127) of head row h of the fp32 partial staged in the
+// V region; the chunk index is swizzled with the row so that the 16 rows
+// written at once by a warp fall on different banks
+__device__ __forceinline__ int stage_off(int h, int c) { return h * kD + ((c ^ (h & 7)) << 2); }
 
 // Raw bytes of one producer item: the codes (32 B) and scales (64 B) of 64
 // dims of one entry.
@@ -209,6 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_slot, kTmemCols);
+  // the block's 64 query rows (64 KB) into L2 now: the softmax warps read them
+  // in two dependent batches while the producers wait for their first rows
+  for (int i = threadIdx.x; i < nh * (kD * 2 / 128); i += kThreads) {
+    const uint16_t* qr = p.q + ((row * p.Hq) + h0 + i / 8) * kD + (i % 8) * 64;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(qr));
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -582,6 +599,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
             }
             dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
           }
+        } else if (p.cluster_merge) {
+          // partial into the idle V region; merged over DSMEM below
+          float* stage = reinterpret_cast<float*>(vs);
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<float4*>(stage + stage_off(h, c0 / 4 + c)) =
+                l_o > 0.0f ? make_float4(f * o[4 * c], f * o[4 * c + 1], f * o[4 * c + 2],
+                                         f * o[4 * c + 3])
+                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         } else {
           float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + c0);
 #pragma unroll
@@ -592,10 +618,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         }
       }
       if (lane < 16 && h < nh) {
+        const float2 ml = make_float2(l_o > 0.0f ? m_o : -INFINITY, l_o);
         if (p.nsplit == 1) {
           if (p.lse) p.lse[row * p.Hq + h0 + h] = l_o > 0.0f ? (m_o + log2f(l_o)) * kLn2 : -INFINITY;
+        } else if (p.cluster_merge) {
+          sm.ml[h] = ml;
         } else {
-          p.ws_ml[slot * kHB + h] = make_float2(l_o > 0.0f ? m_o : -INFINITY, l_o);
+          p.ws_ml[slot * kHB + h] = ml;
         }
       }
     }
@@ -608,6 +637,58 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) record_error(p.err, CSA2_ERR_TIMEOUT);
+
+  if (p.cluster_merge) {
+    // Split s of the cluster merges heads [s share, (s + 1) share) of all splits'
+    // partials: weights 2^(m_s - M) (l_s for the sums), read over DSMEM.
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();                                   // every split's partial is staged
+    const int ns = p.nsplit;
+    const int share = (kHB + ns - 1) / ns;
+    const int hA = split * share, hB = min(nh, hA + share);
+    const int units = max(0, hB - hA) * (kD / 4);
+    for (int u = threadIdx.x; u < units; u += kThreads) {
+      const int hh = hA + u / (kD / 4), c = u % (kD / 4);
+      float mv[8], lv[8];
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r < ns) {
+          const float2 ml = cl.map_shared_rank(&sm.ml[hh], r)[0];
+          mv[r] = ml.x;
+          lv[r] = ml.y;
+          M = fmaxf(M, ml.x);
+        }
+      }
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      float L = 0.0f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          if (r < ns && mv[r] != -INFINITY) {
+            const float w = exp2f(mv[r] - M);
+            const float* st = cl.map_shared_rank(reinterpret_cast<float*>(vs), r);
+            const float4 v = *reinterpret_cast<const float4*>(st + stage_off(hh, c));
+            L += w * lv[r];
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+          }
+        }
+      }
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+      __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+      *reinterpret_cast<uint2*>(p.out + ((row * p.Hq) + h0 + hh) * kD + 4 * c) = pk;
+      if (c == 0 && p.lse)
+        p.lse[row * p.Hq + h0 + hh] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    cl.sync();                                   // no split leaves while others read it
+  }
 }
 
 }  // namespace
@@ -618,7 +699,8 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
-                                  float* ws_o, float2* ws_ml, int* err, cudaStream_t stream) {
+                                  float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
+                                  bool* merged) {
   AttnParams p;
   p.q = q;
   p.kv_packed = kv_packed;
@@ -637,11 +719,40 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
   p.ws_o = ws_o;
   p.ws_ml = ws_ml;
   p.err = err;
+  p.cluster_merge = 0;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(rows, nhb, nsplit);
+  if (merged != nullptr) *merged = false;
+  if (nsplit > 1 && nsplit <= 8 && merged != nullptr) {
+    // the splits of each (row, head block) as one cluster: merged in DSMEM
+    p.cluster_merge = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)nsplit;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, sparse_attn_tc_kernel, &cfg) == cudaSuccess &&
+        nclusters > 0) {
+      e = cudaLaunchKernelEx(&cfg, sparse_attn_tc_kernel, p);
+      if (e == cudaSuccess) {
+        *merged = true;
+        return cudaSuccess;
+      }
+    }
+    (void)cudaGetLastError();   // fall back to partials in the workspace
+    p.cluster_merge = 0;
+  }
   sparse_attn_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }

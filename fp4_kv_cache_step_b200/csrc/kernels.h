@@ -48,12 +48,16 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
                                float* lse, void* workspace, int* err, cudaStream_t stream);
 
-// Tensor-core attention kernel (attn_tc.cu); partials go to ws_o/ws_ml when nsplit > 1.
+// Tensor-core attention kernel (attn_tc.cu). With nsplit > 1 the splits are
+// merged inside the kernel (thread-block clusters, *merged set to true) when
+// `merged` is non-null and the cluster fits; otherwise partials go to
+// ws_o/ws_ml for attn_combine_kernel.
 int sparse_attn_tc_tile();
 cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
-                                  float* ws_o, float2* ws_ml, int* err, cudaStream_t stream);
+                                  float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
+                                  bool* merged);
 
 }  // namespace csa2
