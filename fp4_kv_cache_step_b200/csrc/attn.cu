@@ -21,6 +21,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(const float* __restrict__ ws_o, const float2* __restrict__ ws_ml, int Hq,
                     int nhb, int nsplit, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait_and_release();
   const size_t row = blockIdx.x;
   const int h = blockIdx.y;
   const int hb = h / kHB, r = h % kHB;
@@ -111,9 +112,8 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                         softmax_scale, p.nhb, p.nsplit, p.split_len, out, lse,
                                         ws_o, ws_ml, err, stream, &merged);
   if (e != cudaSuccess || p.nsplit == 1 || merged) return e;
-  attn_combine_kernel<<<dim3(rows, Hq), 128, 0, stream>>>(ws_o, ws_ml, Hq, p.nhb, p.nsplit, out,
-                                                          lse);
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3(rows, Hq), dim3(128), 0, stream, dim3(1), ws_o,
+                    ws_ml, Hq, p.nhb, p.nsplit, out, lse);
 }
 
 }  // namespace csa2

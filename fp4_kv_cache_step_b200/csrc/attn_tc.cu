@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     const uint16_t* qr = p.q + ((row * p.Hq) + h0 + i / 8) * kD + (i % 8) * 64;
     asm volatile("prefetch.global.L2 [%0];" ::"l"(qr));
   }
+  pdl_wait_and_release();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -744,7 +745,8 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, sparse_attn_tc_kernel, &cfg) == cudaSuccess &&
         nclusters > 0) {
-      e = cudaLaunchKernelEx(&cfg, sparse_attn_tc_kernel, p);
+      e = launch_pdl(sparse_attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream,
+                     dim3(1, 1, (unsigned)nsplit), p);
       if (e == cudaSuccess) {
         *merged = true;
         return cudaSuccess;
@@ -753,8 +755,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
     (void)cudaGetLastError();   // fall back to partials in the workspace
     p.cluster_merge = 0;
   }
-  sparse_attn_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(sparse_attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, dim3(1), p);
 }
 
 }  // namespace csa2

@@ -47,4 +47,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch: a kernel launched with the programmatic stream
+// serialisation attribute may start while the previous kernel of the stream is
+// still running. It waits here before touching global memory that kernel may
+// write or read, then lets its own dependents start (which therefore never
+// overlap the kernel before it). Without the attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace csa2

@@ -29,6 +29,7 @@ index_score_simt_kernel(const uint8_t* __restrict__ idx_q, const float* __restri
                         int C, float* __restrict__ scores, int* err) {
   extern __shared__ __align__(16) float qs[];   // [Hi][Di] then w[Hi]
   float* ws = qs + Hi * Di;
+  pdl_wait_and_release();
   const int tile = blockIdx.x;
   const size_t row = (size_t)blockIdx.z * Tq + blockIdx.y;
   const int b = blockIdx.z;
@@ -120,9 +121,8 @@ cudaError_t launch_index_score(const uint8_t* idx_q, const float* idx_w, const u
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(ceil_div(len, kTileEntries), Tq, B);
-  index_score_simt_kernel<<<grid, kTileEntries, smem, stream>>>(idx_q, idx_w, idx_k, Tq, N, Hi, Di,
-                                                                nvalid, cand, C, scores, err);
-  return cudaGetLastError();
+  return launch_pdl(index_score_simt_kernel, grid, dim3(kTileEntries), smem, stream, dim3(1),
+                    idx_q, idx_w, idx_k, Tq, N, Hi, Di, nvalid, cand, C, scores, err);
 }
 
 }  // namespace csa2

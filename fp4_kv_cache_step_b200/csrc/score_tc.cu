@@ -98,6 +98,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   int* scan_tmp = tile_pre + p.G + 1;                                               // [kThreads/32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait_and_release();
 
   // ---- prefix of tile counts over groups (contiguous chunk per thread)
   {
@@ -412,8 +413,8 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
   // upper bound on the tile count; CTAs beyond the real count get empty ranges
   const long long max_tiles = (long long)p.G * ((N + kTileM * p.sub - 1) / (kTileM * p.sub));
   const int grid = (int)std::min<long long>(sm_count(), std::max<long long>(1, max_tiles));
-  index_score_tc_kernel<<<grid, kThreads, smem, stream>>>(kmap, qmap, p);
-  return cudaGetLastError();
+  return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kThreads), smem, stream, dim3(1),
+                    kmap, qmap, p);
 }
 
 }  // namespace csa2

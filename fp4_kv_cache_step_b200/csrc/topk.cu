@@ -324,6 +324,7 @@ topk_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict_
             int32_t* __restrict__ cand_out, int* err) {
   extern __shared__ uint32_t staged[];
   __shared__ Scratch sc;
+  pdl_wait_and_release();
   const size_t row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Row r;
@@ -576,6 +577,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int ld, const int32_t* __r
                     int Cout, int32_t* __restrict__ cand_out, int slice, int* err) {
   extern __shared__ uint32_t keys[];
   __shared__ ClusterShared sc;
+  pdl_wait_and_release();
   cg::cluster_group cl = cg::this_cluster();
   const int cs = (int)cl.num_blocks();
   const int rank = (int)cl.block_rank();
@@ -738,33 +740,20 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * cs), 1, 1);
-    cfg.blockDim = dim3(kCThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, scores, ld, nvalid, cand, K, topk_idx,
-                              Cout, cand_out, slice, err);
+    return launch_pdl(topk_cluster_kernel, dim3((unsigned)(rows * cs)), dim3(kCThreads), smem,
+                      stream, dim3((unsigned)cs, 1, 1), scores, ld, nvalid, cand, K, topk_idx,
+                      Cout, cand_out, slice, err);
   }
   if (ld <= kSmemKeyCap) {
     size_t smem = (size_t)ld * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_kernel<true><<<rows, kThreads, smem, stream>>>(scores, ld, nvalid, cand, K, topk_idx,
-                                                        Cout, cand_out, err);
-  } else {
-    topk_kernel<false><<<rows, kThreads, 0, stream>>>(scores, ld, nvalid, cand, K, topk_idx, Cout,
-                                                      cand_out, err);
+    return launch_pdl(topk_kernel<true>, dim3(rows), dim3(kThreads), smem, stream, dim3(1), scores,
+                      ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
   }
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel<false>, dim3(rows), dim3(kThreads), 0, stream, dim3(1), scores, ld,
+                    nvalid, cand, K, topk_idx, Cout, cand_out, err);
 }
 
 }  // namespace csa2
