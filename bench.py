@@ -307,40 +307,68 @@ def run_ours(args):
 
 
 def run_e2e(args, w, dw, flush, csa2, torch):
-    """Same step through the public call, with this step's query-side inputs
-    copied from pinned host memory and the outputs copied back, all inside the
-    timed region. The FP4 cache and indexer keys stay resident (they are the
-    cache)."""
+    """The metric through the public call, end to end: every step copies its
+    query-side inputs (queries, indexer queries and weights, lengths) from pinned
+    host memory, runs csa2_layer_step, and copies the attention output and lse
+    back to pinned host memory. The FP4 cache and the indexer keys stay resident
+    (they are the cache; 402 MB, larger than L2). Steps are issued round-robin on
+    three streams with their own buffers, as a serving loop would, so one step's
+    copies overlap another's kernels; the value is steps / elapsed device time
+    from the first timed step's start to the last one's end."""
     from fp4_kv_cache_step_b200 import workloads as wl
-    stream = torch.cuda.current_stream()
+    nslot = 3
+    dev = dw.idx_k.device
     host_in = {
         "q": torch.from_numpy(wl.q(w, 0).view(np.int16)).view(torch.bfloat16).pin_memory(),
         "idx_q": torch.from_numpy(wl.idx_q(w, 0)).pin_memory(),
         "idx_w": torch.from_numpy(wl.idx_w(w, 0)).pin_memory(),
         "nvalid": torch.from_numpy(wl.nvalid(w)).pin_memory(),
     }
-    dev_in = {"q": dw.q[0], "idx_q": dw.idx_q[0], "idx_w": dw.idx_w[0], "nvalid": dw.nvalid}
-    host_out = torch.empty(dw.out[0].shape, dtype=torch.bfloat16).pin_memory()
-    host_lse = torch.empty(dw.lse[0].shape, dtype=torch.float32).pin_memory()
+    slots = []
+    for _ in range(nslot):
+        d = {k: torch.empty_like(t, device=dev) for k, t in host_in.items()}
+        d["topk"] = torch.full_like(dw.topk, -1)
+        d["out"] = torch.empty_like(dw.out[0])
+        d["lse"] = torch.empty_like(dw.lse[0])
+        d["host_out"] = torch.empty(d["out"].shape, dtype=torch.bfloat16).pin_memory()
+        d["host_lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
+        d["shared"] = csa2.Csa2Shared(dw.kv_packed, dw.kv_scale, dw.idx_k, d["topk"], None)
+        d["args"] = csa2.layer_args(d["q"], d["nvalid"], d["out"], w.K, w.softmax_scale,
+                                    idx_q=d["idx_q"], idx_w=d["idx_w"], lse=d["lse"], N=w.N)
+        need = csa2.layer_step_workspace_bytes(wl.FULL, d["args"], d["shared"])
+        d["ws"] = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        d["stream"] = torch.cuda.Stream(device=dev)
+        slots.append(d)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_out.numel() * 2 + host_lse.numel() * 4
-    times = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xff)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for k, t in host_in.items():
-            dev_in[k].copy_(t, non_blocking=True)
-        dw.step(layers=[0])
-        host_out.copy_(dw.out[0], non_blocking=True)
-        host_lse.copy_(dw.lse[0], non_blocking=True)
-        b.record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            times.append(a.elapsed_time(b))
-    ms = statistics.mean(times)
+    d2h = slots[0]["host_out"].numel() * 2 + slots[0]["host_lse"].numel() * 4
+
+    def one_step(d):
+        with torch.cuda.stream(d["stream"]):
+            for k, t in host_in.items():
+                d[k].copy_(t, non_blocking=True)
+            csa2.csa2_layer_step(wl.FULL, d["args"], d["shared"], d["ws"])
+            d["host_out"].copy_(d["out"], non_blocking=True)
+            d["host_lse"].copy_(d["lse"], non_blocking=True)
+
+    for i in range(args.warmup):
+        one_step(slots[i % nslot])
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    start.record(torch.cuda.current_stream())
+    for d in slots:
+        d["stream"].wait_event(start)
+    for i in range(args.steps):
+        one_step(slots[i % nslot])
+    ends = []
+    for d in slots:
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(d["stream"])
+        ends.append(e)
+    torch.cuda.synchronize()
+    ms = max(start.elapsed_time(e) for e in ends) / args.steps
     return {"value": 1e3 / ms, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "streams": nslot,
+            "l2": "not flushed: the resident cache (402 MB) is larger than L2"}
 
 
 # --------------------------------------------------------------- CPU oracle
