@@ -241,9 +241,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     const uint8_t* sc_b = p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
     const int32_t* topk_row = p.topk + row * p.K;
 
-    auto load_index = [&](int t) -> int {
+    // index of entry e of tile t, as loaded (checked later: the check waits
+    // for the load, so it runs a tile after the load was issued)
+    auto fetch_index = [&](int t) -> int {
       const int kk = k_begin + t * kT + e;
-      int id = (t < nt && kk < k_end) ? __ldg(topk_row + kk) : -1;
+      return (t < nt && kk < k_end) ? __ldg(topk_row + kk) : -1;
+    };
+    auto check_index = [&](int id) -> int {
       if (id >= p.N || id < -1) {
         record_error(p.err, CSA2_ERR_DEVICE_INDEX);
         id = -1;
@@ -284,17 +288,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       }
     };
 
-    // indices and L2 prefetch two tiles ahead, raw bytes one tile ahead
-    int id_cur = load_index(0);
-    int id_next = load_index(1);
+    // Indices loaded three tiles ahead (and checked a tile later, when the load
+    // has landed), rows prefetched into L2 two tiles ahead, raw bytes loaded one
+    // tile ahead: nothing on a producer's path waits for a load it just issued.
+    int id_cur = check_index(fetch_index(0));
+    int id_next = check_index(fetch_index(1));
+    int id_after = check_index(fetch_index(2));
+    int id_far = fetch_index(3);
     prefetch_rows(id_cur);
     prefetch_rows(id_next);
+    prefetch_rows(id_after);
     Raw raw[2];
     load_raw(id_cur, raw);
     bool go = true;
     for (int t = 0; go && t < nt; ++t) {
       const int buf = t & 1;
-      const int id_after = load_index(t + 2);
       // the buffer (and its valid bits) is free once P(t-2) V(t-2) has completed
       if (!mbar_wait_warp(&sm.bar.v_free[buf], ((t >> 1) & 1) ^ 1, abort_flag)) {
         go = false;
@@ -321,9 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.v_full[buf]);
-      prefetch_rows(id_after);
+      const int id_far_checked = check_index(id_far);
+      prefetch_rows(id_far_checked);
+      id_far = fetch_index(t + 4);
       id_cur = id_next;
       id_next = id_after;
+      id_after = id_far_checked;
       load_raw(id_cur, raw);
     }
   } else if (warp == kMmaWarp) {
