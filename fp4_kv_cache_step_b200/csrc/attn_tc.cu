@@ -67,6 +67,7 @@ struct Smem {
   uint32_t tmem_slot;
   int abort_flag;
   uint32_t valid[2][kT / 32];   // bit i of word w: entry 32 w + i of the tile is selected
+                                // (byte w of a buffer written by producer warp w)
   float head_scale[kHB];
   float2 ml[kHB];               // this split's (reference maximum, row sum) per head
 };
@@ -179,11 +180,11 @@ struct AttnParams {
 // written at once by a warp fall on different banks
 __device__ __forceinline__ int stage_off(int h, int c) { return h * kD + ((c ^ (h & 7)) << 2); }
 
-// Raw bytes of one producer item: the codes (32 B) and scales (64 B) of 64
-// dims of one entry.
+// Raw bytes a producer lane holds for one entry: the codes (8 B) and scales
+// (16 B) of dims 16u .. 16u+15 and of dims 256+16u .. 256+16u+15.
 struct Raw {
-  uint4 c[2];
-  uint4 s[4];
+  uint2 c[2];
+  uint4 s[2];
 };
 
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnParams p) {
@@ -234,18 +235,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
 
   if (warp < kProducerWarps) {
     // ------------------------------------------------------------ gather + dequantise
-    const int tid = threadIdx.x;          // 0..255
-    const int e = tid & (kT - 1);         // entry of the tile this thread gathers
-    const int apair = tid >> 6;           // atoms 2 apair, 2 apair + 1
+    // Warp w gathers entries 8w .. 8w+7 of every tile, two per round: lane
+    // 16 j + u takes dims 16u .. 16u+15 and 256+16u .. 256+16u+15 of entry
+    // 8w + 2r + j, so each load of a warp covers whole 128-byte lines of two
+    // rows (one line of codes or two of scales per row) instead of 32 rows.
+    const int u = lane & 15, half = lane >> 4;
     const uint8_t* pk_b = p.kv_packed + (size_t)b * p.N * (kD / 2);
     const uint8_t* sc_b = p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
     const int32_t* topk_row = p.topk + row * p.K;
 
-    // index of entry e of tile t, as loaded (checked later: the check waits
-    // for the load, so it runs a tile after the load was issued)
+    // lanes 0-7: index of entry 8w + lane of tile t, as loaded (checked later:
+    // the check waits for the load, so it runs a tile after the load was issued)
     auto fetch_index = [&](int t) -> int {
-      const int kk = k_begin + t * kT + e;
-      return (t < nt && kk < k_end) ? __ldg(topk_row + kk) : -1;
+      const int kk = k_begin + t * kT + warp * 8 + lane;
+      return (lane < 8 && t < nt && kk < k_end) ? __ldg(topk_row + kk) : -1;
     };
     auto check_index = [&](int id) -> int {
       if (id >= p.N || id < -1) {
@@ -254,36 +257,36 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       }
       return id;
     };
-    // L2 prefetch of a row: thread groups 0-1 the packed row, groups 2-3 the scale row
-    auto prefetch_rows = [&](int id) {
+    // L2 prefetch of the warp's 8 rows: lane 4 j + q, q = 0, 1, half of the
+    // packed row of entry j; q = 2, 3, half of its scale row
+    auto prefetch_rows = [&](int ids) {
+      const int id = __shfl_sync(0xffffffffu, ids, lane >> 2);
       if (id >= 0) {
-        if (apair < 2) {
-          const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + apair * 128;
+        const int q = lane & 3;
+        if (q < 2) {
+          const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + q * 128;
           asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(pr));
         } else {
-          const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + (apair - 2) * 256;
+          const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + (q - 2) * 256;
           asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(sr));
           asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(sr + 128));
         }
       }
     };
-    // item i (0, 1): atom 2 apair + i of entry e
-    auto load_raw = [&](int id, Raw (&r)[2]) {
+    auto load_raw = [&](int ids, Raw (&r)[4]) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int a = 2 * apair + i;
+      for (int rr = 0; rr < 4; ++rr) {
+        const int id = __shfl_sync(0xffffffffu, ids, 2 * rr + half);
         if (id >= 0) {
-          const uint4* pc = reinterpret_cast<const uint4*>(pk_b + (size_t)id * (kD / 2) + a * 32);
-          const uint4* psc =
-              reinterpret_cast<const uint4*>(sc_b + (size_t)(id / kBlockEntries) * kD + a * 64);
-          r[i].c[0] = __ldg(pc);
-          r[i].c[1] = __ldg(pc + 1);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) r[i].s[j] = __ldg(psc + j);
+          const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + 8 * u;
+          const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + 16 * u;
+          r[rr].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
+          r[rr].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
+          r[rr].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
+          r[rr].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
         } else {
-          r[i].c[0] = r[i].c[1] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) r[i].s[j] = make_uint4(0, 0, 0, 0);
+          r[rr].c[0] = r[rr].c[1] = make_uint2(0, 0);
+          r[rr].s[0] = r[rr].s[1] = make_uint4(0, 0, 0, 0);
         }
       }
     };
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     prefetch_rows(id_cur);
     prefetch_rows(id_next);
     prefetch_rows(id_after);
-    Raw raw[2];
+    Raw raw[4];
     load_raw(id_cur, raw);
     bool go = true;
     for (int t = 0; go && t < nt; ++t) {
@@ -308,22 +311,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         go = false;
         break;
       }
-      if (apair == 0) {
-        const uint32_t vb = __ballot_sync(0xffffffffu, id_cur >= 0);
-        if (lane == 0) sm.valid[buf][warp] = vb;
-      }
+      const uint32_t vb = __ballot_sync(0xffffffffu, id_cur >= 0);   // lanes 8-31 hold -1
+      if (lane == 0) reinterpret_cast<uint8_t*>(sm.valid[buf])[warp] = (uint8_t)vb;
       uint8_t* tile = vs + buf * kVTile;
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        uint8_t* dst = tile + (2 * apair + i) * kAtom;
+      for (int rr = 0; rr < 4; ++rr) {
+        const int e = warp * 8 + 2 * rr + half;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 cw = raw[i].c[c >> 2];
-          const uint32_t codes = (c & 3) == 0 ? cw.x : (c & 3) == 1 ? cw.y : (c & 3) == 2 ? cw.z : cw.w;
-          const uint4 sw = raw[i].s[c >> 1];
-          const uint32_t s_lo = (c & 1) ? sw.z : sw.x;
-          const uint32_t s_hi = (c & 1) ? sw.w : sw.y;
-          *reinterpret_cast<uint4*>(dst + swz(e, c)) = dq8(codes, s_lo, s_hi);
+        for (int hh = 0; hh < 2; ++hh) {
+          // dims 256 hh + 16 u .. + 15: atom 4 hh + u / 4, chunks 2 (u % 4) and 2 (u % 4) + 1;
+          // the two rows of a store differ in parity, so its 32 lanes cover
+          // all eight 16-byte bank groups four times
+          uint8_t* dst = tile + (4 * hh + (u >> 2)) * kAtom;
+          const int c = (u & 3) * 2;
+          const uint2 cw = raw[rr].c[hh];
+          const uint4 sw = raw[rr].s[hh];
+          *reinterpret_cast<uint4*>(dst + swz(e, c)) = dq8(cw.x, sw.x, sw.y);
+          *reinterpret_cast<uint4*>(dst + swz(e, c + 1)) = dq8(cw.y, sw.z, sw.w);
         }
       }
       fence_async_smem();
