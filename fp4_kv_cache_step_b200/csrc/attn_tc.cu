@@ -180,6 +180,16 @@ struct AttnParams {
 // written at once by a warp fall on different banks
 __device__ __forceinline__ int stage_off(int h, int c) { return h * kD + ((c ^ (h & 7)) << 2); }
 
+// 64 columns c0 .. c0 + 63 of head row h of a split's partial O, times f, into
+// the fp32 staging area (the idle V region) that the cluster merge reads
+__device__ __forceinline__ void stage_partial64(float* stage, int h, int c0, const float (&o)[64],
+                                                float f) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c)
+    *reinterpret_cast<float4*>(stage + stage_off(h, c0 / 4 + c)) =
+        make_float4(f * o[4 * c], f * o[4 * c + 1], f * o[4 * c + 2], f * o[4 * c + 3]);
+}
+
 // Raw bytes a producer lane holds for one entry: the codes (8 B) and scales
 // (16 B) of dims 16u .. 16u+15 and of dims 256+16u .. 256+16u+15.
 struct Raw {
@@ -340,6 +350,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       id_next = id_after;
       id_after = id_far_checked;
       load_raw(id_cur, raw);
+    }
+    if (p.cluster_merge && go) {
+      // Staging of the split's partial for the merge, shared with the softmax
+      // warps: producer warps q and q + 4 take columns 192 (w >> 2) .. + 191 of
+      // the 16 O rows of TMEM quadrant q (heads 16 q ..), the softmax warp of
+      // the quadrant the last 128. x 2^8 undoes the factor the dequantised
+      // values carry; an empty split is skipped by the merge, whatever it stages.
+      if (mbar_wait_warp(&sm.bar.o_full, 0, abort_flag)) {
+        tc_fence_after();
+        const int quad = warp & 3;
+        const int hq = quad * 16 + (lane & 15);
+        const uint32_t la = (uint32_t)(quad * 32) << 16;
+#pragma unroll 1
+        for (int k = 0; k < 3; ++k) {
+          const int c0 = (warp >> 2) * 192 + k * 64;
+          float o[64];
+          tmem_ld_64(tmem + la + c0, o);
+          if (lane < 16 && hq < nh) stage_partial64(reinterpret_cast<float*>(vs), hq, c0, o, 256.0f);
+        }
+      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -598,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       // nothing selected writes zeros whatever the accumulator holds
       const float f = l_o > 0.0f ? (p.nsplit == 1 ? 256.0f / l_o : 256.0f) : 0.0f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 64) {
+      for (int c0 = p.cluster_merge ? 384 : 0; c0 < kD; c0 += 64) {
         float o[64];
         tmem_ld_64(tmem + lane_addr + c0, o);
         if (!o_owner) continue;
@@ -617,13 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           }
         } else if (p.cluster_merge) {
           // partial into the idle V region; merged over DSMEM below
-          float* stage = reinterpret_cast<float*>(vs);
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<float4*>(stage + stage_off(h, c0 / 4 + c)) =
-                l_o > 0.0f ? make_float4(f * o[4 * c], f * o[4 * c + 1], f * o[4 * c + 2],
-                                         f * o[4 * c + 3])
-                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          stage_partial64(reinterpret_cast<float*>(vs), h, c0, o, 256.0f);
         } else {
           float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + c0);
 #pragma unroll
@@ -656,19 +680,25 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
 
   if (p.cluster_merge) {
     // Split s of the cluster merges heads [s share, (s + 1) share) of all splits'
-    // partials: weights 2^(m_s - M) (l_s for the sums), read over DSMEM.
+    // partials, read over DSMEM: out = sum_r w_r O_r with w_r = 2^(m_r - M) / L,
+    // L = sum_r 2^(m_r - M) l_r, M = max_r m_r. The weights of a head are
+    // computed once (into the idle Q region); then every thread loads its
+    // outputs' partials from all splits before combining them.
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();                                   // every split's partial is staged
     const int ns = p.nsplit;
     const int share = (kHB + ns - 1) / ns;
     const int hA = split * share, hB = min(nh, hA + share);
-    const int units = max(0, hB - hA) * (kD / 4);
-    for (int u = threadIdx.x; u < units; u += kThreads) {
-      const int hh = hA + u / (kD / 4), c = u % (kD / 4);
+    const int nhm = max(0, hB - hA);
+    float* wts = reinterpret_cast<float*>(qs);   // [head - hA][8 splits]
+    for (int i = threadIdx.x; i < nhm; i += kThreads) {
+      const int hh = hA + i;
       float mv[8], lv[8];
       float M = -INFINITY;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
+        mv[r] = -INFINITY;
+        lv[r] = 0.0f;
         if (r < ns) {
           const float2 ml = cl.map_shared_rank(&sm.ml[hh], r)[0];
           mv[r] = ml.x;
@@ -676,32 +706,59 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           M = fmaxf(M, ml.x);
         }
       }
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      float w[8];
       float L = 0.0f;
-      if (M != -INFINITY) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        w[r] = mv[r] != -INFINITY ? exp2f(mv[r] - M) : 0.0f;
+        L += w[r] * lv[r];
+      }
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) wts[i * 8 + r] = w[r] * inv;
+      if (p.lse) p.lse[row * p.Hq + h0 + hh] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+    __syncthreads();
+    const int units = nhm * (kD / 4);
+    constexpr int kBatch = 2;                    // outputs per thread whose loads are in flight together
+#pragma unroll 1
+    for (int base = threadIdx.x; base < units; base += kBatch * kThreads) {
+      float4 v[kBatch][8];
+      float wv[kBatch][8];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int u = base + j * kThreads;
+        const int i = u / (kD / 4), c = u % (kD / 4);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          if (r < ns && mv[r] != -INFINITY) {
-            const float w = exp2f(mv[r] - M);
+          wv[j][r] = (u < units && r < ns) ? wts[i * 8 + r] : 0.0f;
+          v[j][r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (wv[j][r] != 0.0f) {
             const float* st = cl.map_shared_rank(reinterpret_cast<float*>(vs), r);
-            const float4 v = *reinterpret_cast<const float4*>(st + stage_off(hh, c));
-            L += w * lv[r];
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
+            v[j][r] = *reinterpret_cast<const float4*>(st + stage_off(hA + i, c));
           }
         }
       }
-      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-      __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-      *reinterpret_cast<uint2*>(p.out + ((row * p.Hq) + h0 + hh) * kD + 4 * c) = pk;
-      if (c == 0 && p.lse)
-        p.lse[row * p.Hq + h0 + hh] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int u = base + j * kThreads;
+        if (u >= units) break;
+        const int i = u / (kD / 4), c = u % (kD / 4);
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          acc.x = fmaf(wv[j][r], v[j][r].x, acc.x);
+          acc.y = fmaf(wv[j][r], v[j][r].y, acc.y);
+          acc.z = fmaf(wv[j][r], v[j][r].z, acc.z);
+          acc.w = fmaf(wv[j][r], v[j][r].w, acc.w);
+        }
+        __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+        *reinterpret_cast<uint2*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 4 * c) = pk;
+      }
     }
     cl.sync();                                   // no split leaves while others read it
   }
