@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
         L.or_bf16_value.argtypes = [ctypes.c_uint16]
         L.or_fp4_kv_pack.argtypes = [P, I, I, I, P, P]
         L.or_fp4_kv_unpack.argtypes = [P, P, I, I, I, P]
+        L.or_fp4_kv_pack_g16.argtypes = [P, I, I, I, P]
+        L.or_fp4_kv_unpack_g16.argtypes = [P, I, I, I, P]
+        L.or_fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P]
+        L.or_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, D, P, P]
         L.or_index_score.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
         L.or_topk.argtypes = [P, I, I, P, P, I, P]
         L.or_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, P]
@@ -68,7 +72,8 @@ def lib() -> ctypes.CDLL:
         L.or_layer_step.argtypes = [I, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, D,
                                     P, P, P, P]
         for f in (L.or_fp4_kv_pack, L.or_fp4_kv_unpack, L.or_index_score, L.or_topk,
-                  L.or_sparse_attn, L.or_dense_attn, L.or_layer_step):
+                  L.or_sparse_attn, L.or_dense_attn, L.or_layer_step, L.or_fp4_kv_pack_g16,
+                  L.or_fp4_kv_unpack_g16, L.or_fp4_kv_append_g16, L.or_sparse_attn_g16):
             f.restype = I
         _lib = L
     return _lib
@@ -135,6 +140,63 @@ def fp4_kv_unpack(packed: np.ndarray, scale: np.ndarray) -> np.ndarray:
     _check(lib().or_fp4_kv_unpack(_ptr(packed), _ptr(scale), B, N, D, _ptr(out)),
            "or_fp4_kv_unpack")
     return out
+
+
+# ---------------------------------------------------------------- FP4 KV, 16-channel scales
+GROUP_CHANNELS = 16
+
+
+def g16_row_bytes(D: int) -> int:
+    """Bytes of one entry in the pages' layout: D/2 code bytes, then D/16 scales."""
+    return D // 2 + D // GROUP_CHANNELS
+
+
+def fp4_kv_pack_g16(kv: np.ndarray) -> np.ndarray:
+    """kv float32 [B][N][D] -> rows u8 [B][N][D/2 + D/16] (one E4M3 scale per 16
+    channels of an entry, after its codes)."""
+    kv = _c(kv, np.float32)
+    B, N, D = kv.shape
+    rows = np.zeros((B, N, g16_row_bytes(D)), np.uint8)
+    _check(lib().or_fp4_kv_pack_g16(_ptr(kv), B, N, D, _ptr(rows)), "or_fp4_kv_pack_g16")
+    return rows
+
+
+def fp4_kv_unpack_g16(rows: np.ndarray, D: int) -> np.ndarray:
+    rows = _c(rows, np.uint8)
+    B, N, rb = rows.shape
+    assert rb == g16_row_bytes(D)
+    out = np.zeros((B, N, D), np.float64)
+    _check(lib().or_fp4_kv_unpack_g16(_ptr(rows), B, N, D, _ptr(out)), "or_fp4_kv_unpack_g16")
+    return out
+
+
+def fp4_kv_append_g16(rows: np.ndarray, kv_new: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """A copy of `rows` with kv_new[b][t] (float32 [B][T][D]) quantised into
+    row pos[b][t]."""
+    out = np.array(rows, dtype=np.uint8, copy=True, order="C")
+    kv_new = _c(kv_new, np.float32)
+    pos = _c(pos, np.int32)
+    B, T, D = kv_new.shape
+    N = out.shape[1]
+    _check(lib().or_fp4_kv_append_g16(_ptr(kv_new), _ptr(pos), B, T, N, D, _ptr(out)),
+           "or_fp4_kv_append_g16")
+    return out
+
+
+def sparse_attn_g16(q_bf16, rows, idx, softmax_scale):
+    """Sparse attention over a cache in the 16-channel layout; as sparse_attn."""
+    q_bf16 = _c(q_bf16, np.uint16)
+    rows = _c(rows, np.uint8)
+    idx = _c(idx, np.int32)
+    B, Tq, Hq, D = q_bf16.shape
+    N = rows.shape[1]
+    K = idx.shape[2]
+    out = np.zeros((B, Tq, Hq, D), np.float64)
+    lse = np.zeros((B, Tq, Hq), np.float64)
+    _check(lib().or_sparse_attn_g16(_ptr(q_bf16), _ptr(rows), _ptr(idx), B, Tq, Hq, D, N, K,
+                                    float(softmax_scale), _ptr(out), _ptr(lse)),
+           "or_sparse_attn_g16")
+    return out, lse
 
 
 # ---------------------------------------------------------------- indexer

@@ -160,6 +160,94 @@ int or_fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale,
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP4 main KV in the pages' own layout: one E4M3 scale per 16 channels of    */
+/* an entry, no second-level scale ("Detailed Notes On DeepSeek V4 Point 1    */
+/* Flash In Simple Words", "FP4 Main KV Cache To Halve Storage Again"; the    */
+/* mengman.github.io interpretation, 3.5). An entry row holds its D/2 code     */
+/* bytes followed by its D/16 scale bytes. The scale of a group follows the   */
+/* same reading as the block layout: E4M3 (nearest, ties even) of max|x|/6.   */
+/* ------------------------------------------------------------------------ */
+
+#define OR_GROUP 16
+
+static size_t g16_row_bytes(int D) { return (size_t)D / 2 + (size_t)D / OR_GROUP; }
+
+/* Quantise one entry of D values into its row. */
+static int g16_quantise_row(const float* x, int D, uint8_t* row) {
+    for (int g = 0; g < D / OR_GROUP; ++g) {
+        double amax = 0.0;
+        for (int i = 0; i < OR_GROUP; ++i) {
+            float v = x[g * OR_GROUP + i];
+            if (!isfinite(v)) return OR_NONFINITE;
+            if (fabs((double)v) > amax) amax = fabs((double)v);
+        }
+        uint8_t sc = or_e4m3_from_double(amax / 6.0);
+        row[D / 2 + g] = sc;
+        double s = or_e4m3_value(sc);
+        for (int i = 0; i < OR_GROUP; ++i) {
+            int c = g * OR_GROUP + i;
+            uint8_t code = or_e2m1_code((double)x[c], s);
+            uint8_t* byte = &row[c / 2];
+            if (c % 2 == 0)
+                *byte = (uint8_t)((*byte & 0xF0) | code);
+            else
+                *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+        }
+    }
+    return OR_OK;
+}
+
+static int g16_shape_ok(int B, int N, int D) {
+    return B >= 0 && N >= 0 && D > 0 && D % OR_GROUP == 0;
+}
+
+int or_fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8_t* kv_rows) {
+    if (!kv || !kv_rows || !g16_shape_ok(B, N, D)) return OR_BAD_ARG;
+    const size_t rb = g16_row_bytes(D);
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n) {
+            int rc = g16_quantise_row(kv + ((size_t)b * N + n) * D, D,
+                                      kv_rows + ((size_t)b * N + n) * rb);
+            if (rc != OR_OK) return rc;
+        }
+    return OR_OK;
+}
+
+/* Appending new entries: entry t of row b is quantised into position
+ * pos[b][t] of the cache; no other row changes (each row carries its own
+ * scales). */
+int or_fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, int T, int N, int D,
+                         uint8_t* kv_rows) {
+    if (!kv_new || !pos || !kv_rows || !g16_shape_ok(B, N, D) || T < 0) return OR_BAD_ARG;
+    const size_t rb = g16_row_bytes(D);
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            int32_t n = pos[(size_t)b * T + t];
+            if (n < 0 || n >= N) return OR_BAD_INDEX;
+            int rc = g16_quantise_row(kv_new + ((size_t)b * T + t) * D, D,
+                                      kv_rows + ((size_t)b * N + n) * rb);
+            if (rc != OR_OK) return rc;
+        }
+    return OR_OK;
+}
+
+static double g16_value(const uint8_t* kv_rows, int N, int D, int b, int n, int c) {
+    const uint8_t* row = kv_rows + ((size_t)b * N + n) * g16_row_bytes(D);
+    uint8_t byte = row[c / 2];
+    uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    return or_e2m1_value(code) * or_e4m3_value(row[D / 2 + c / OR_GROUP]);
+}
+
+int or_fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, double* out) {
+    if (!kv_rows || !out || !g16_shape_ok(B, N, D)) return OR_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        for (int n = 0; n < N; ++n)
+            for (int c = 0; c < D; ++c)
+                out[((size_t)b * N + n) * D + c] = g16_value(kv_rows, N, D, b, n, c);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Indexer score: s_j = sum_h w_h * ReLU(q_h . k_j).                          */
 /* ------------------------------------------------------------------------ */
 
@@ -278,13 +366,22 @@ int or_topk(const double* scores, int rows, int ld,
 /* Sparse softmax attention over the selected rows; K doubles as V.          */
 /* ------------------------------------------------------------------------ */
 
-int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
-                   const int32_t* topk, int B, int Tq, int Hq, int D, int N, int K,
-                   double softmax_scale, double* out, double* lse) {
-    if (!q || !kv_packed || !kv_scale || !topk || !out || B < 0 || Tq < 0 || Hq <= 0 ||
-        D <= 0 || N < 0 || K <= 0)
-        return OR_BAD_ARG;
-    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+/* Dequantised value of channel c of entry n of row b, for either layout. */
+typedef struct {
+    const uint8_t* kv_packed;   /* block layout: codes; 16-channel layout: rows */
+    const uint8_t* kv_scale;    /* block layout: scales; NULL for the 16-channel layout */
+    int N, D;
+} kv_source;
+
+static double kv_source_value(const kv_source* src, int b, int n, int c) {
+    if (src->kv_scale)
+        return kv_value(src->kv_packed, src->kv_scale, src->N, src->D, b, n, c);
+    return g16_value(src->kv_packed, src->N, src->D, b, n, c);
+}
+
+static int sparse_attn_rows(const uint16_t* q, const kv_source* src, const int32_t* topk,
+                            int B, int Tq, int Hq, int D, int N, int K,
+                            double softmax_scale, double* out, double* lse) {
     double* v = (double*)malloc(sizeof(double) * (size_t)K * D);
     double* logit = (double*)malloc(sizeof(double) * (size_t)K);
     if (!v || !logit) { free(v); free(logit); return OR_BAD_ARG; }
@@ -299,7 +396,7 @@ int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* k
                 if (id < 0) continue;
                 if (id >= N) { rc = OR_BAD_INDEX; break; }
                 for (int c = 0; c < D; ++c)
-                    v[(size_t)n * D + c] = kv_value(kv_packed, kv_scale, N, D, b, id, c);
+                    v[(size_t)n * D + c] = kv_source_value(src, b, id, c);
                 ++n;
             }
             if (rc != OR_OK) break;
@@ -335,6 +432,27 @@ int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* k
     free(v);
     free(logit);
     return rc;
+}
+
+int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                   const int32_t* topk, int B, int Tq, int Hq, int D, int N, int K,
+                   double softmax_scale, double* out, double* lse) {
+    if (!q || !kv_packed || !kv_scale || !topk || !out || B < 0 || Tq < 0 || Hq <= 0 ||
+        D <= 0 || N < 0 || K <= 0)
+        return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    kv_source src = {kv_packed, kv_scale, N, D};
+    return sparse_attn_rows(q, &src, topk, B, Tq, Hq, D, N, K, softmax_scale, out, lse);
+}
+
+int or_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows, const int32_t* topk,
+                       int B, int Tq, int Hq, int D, int N, int K,
+                       double softmax_scale, double* out, double* lse) {
+    if (!q || !kv_rows || !topk || !out || Tq < 0 || Hq <= 0 || K <= 0 ||
+        !g16_shape_ok(B, N, D))
+        return OR_BAD_ARG;
+    kv_source src = {kv_rows, NULL, N, D};
+    return sparse_attn_rows(q, &src, topk, B, Tq, Hq, D, N, K, softmax_scale, out, lse);
 }
 
 int or_dense_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,

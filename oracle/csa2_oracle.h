@@ -19,7 +19,9 @@
  * shared key per entry; one E4M3 scale per channel per 64-entry block equal to
  * round_e4m3(blockmax / 6); E2M1 codes by round-to-nearest-even on the E2M1
  * grid, saturating at 6; top-K ranked by (score descending, index ascending),
- * emitted ascending by index and padded with -1.
+ * emitted ascending by index and padded with -1. For the pages' own layout
+ * (one E4M3 scale per 16 channels of an entry) the same scale rule is applied
+ * per group, and an entry's scale bytes follow its code bytes in one row.
  *
  * All functions return 0 on success and a nonzero code on a bad argument or a
  * non-finite value, never abort. Every pointer is host memory owned by the
@@ -27,6 +29,7 @@
  *   kv           float [B][N][D]
  *   kv_packed    u8    [B][N][D/2]     low nibble = even channel
  *   kv_scale     u8    [B][N/64][D]    E4M3 bytes
+ *   kv_rows      u8    [B][N][D/2 + D/16]  16-channel layout: codes, then scales
  *   q            u16   [B][Tq][Hq][D]  bf16 bit patterns
  *   idx_q        u8    [B][Tq][Hi][Di] E4M3 bytes
  *   idx_w        float [B][Tq][Hi]
@@ -64,6 +67,15 @@ int or_fp4_kv_pack(const float* kv, int B, int N, int D,
 int or_fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale,
                      int B, int N, int D, double* out);
 
+/* The pages' own FP4 layout: one E4M3 scale per 16 channels of an entry.
+ * kv_rows[b][n] = D/2 code bytes (channel c in byte c/2, low nibble = even c)
+ * followed by D/16 scale bytes; scale = E4M3(max |x| of the group / 6). */
+int or_fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8_t* kv_rows);
+int or_fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, double* out);
+/* Quantise kv_new[b][t] into row pos[b][t] of kv_rows; other rows unchanged. */
+int or_fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, int T, int N, int D,
+                         uint8_t* kv_rows);
+
 /* scores[b][t][j] for j < nvalid[b][t] (cand == NULL), or scores[b][t][i] for
  * candidate i (cand != NULL); positions with no valid entry get -infinity.
  * The output row length is N without a pool and C with one. */
@@ -84,6 +96,11 @@ int or_topk(const double* scores, int rows, int ld,
 int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
                    const int32_t* topk, int B, int Tq, int Hq, int D, int N, int K,
                    double softmax_scale, double* out, double* lse);
+
+/* Sparse attention over a cache in the 16-channel-scale layout. */
+int or_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows, const int32_t* topk,
+                       int B, int Tq, int Hq, int D, int N, int K,
+                       double softmax_scale, double* out, double* lse);
 
 /* Softmax attention of every head over all entries j < nvalid[b][t] (dense). */
 int or_dense_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
