@@ -48,7 +48,8 @@ class LayerArgs(ctypes.Structure):
 EXPORTS = ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk",
            "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn",
            "csa2_layer_step_workspace_bytes", "csa2_layer_step", "csa2_check_device_errors",
-           "csa2_last_error", "csa2_sparse_attn_noalloc")
+           "csa2_last_error", "csa2_sparse_attn_noalloc", "fp4_kv_pack_g16", "fp4_kv_unpack_g16",
+           "fp4_kv_append_g16", "csa2_sparse_attn_g16")
 
 _lib = None
 
@@ -71,6 +72,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.csa2_sparse_attn_workspace_bytes.restype = Z
     L.csa2_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
     L.csa2_sparse_attn_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, F, P, P, P]
+    L.fp4_kv_pack_g16.argtypes = [P, I, I, I, P, P]
+    L.fp4_kv_unpack_g16.argtypes = [P, I, I, I, P, P]
+    L.fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P, P]
+    L.csa2_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
     L.csa2_layer_step_workspace_bytes.argtypes = [ctypes.POINTER(LayerArgs), I,
                                                   ctypes.POINTER(SharedState)]
     L.csa2_layer_step_workspace_bytes.restype = Z
@@ -79,7 +84,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.csa2_last_error.argtypes = []
     L.csa2_last_error.restype = ctypes.c_char_p
     for f in ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk", "csa2_sparse_attn",
-              "csa2_layer_step", "csa2_check_device_errors", "csa2_sparse_attn_noalloc"):
+              "csa2_layer_step", "csa2_check_device_errors", "csa2_sparse_attn_noalloc",
+              "fp4_kv_pack_g16", "fp4_kv_unpack_g16", "fp4_kv_append_g16", "csa2_sparse_attn_g16"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -140,6 +146,46 @@ def fp4_kv_unpack(packed: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
     _check(load().fp4_kv_unpack(_p(packed), _p(scale), B, N, 2 * Dh, _p(out),
                                 _stream(packed.device)), "fp4_kv_unpack")
     return out
+
+
+# ------------------------------------------------------------------- FP4 KV, 16-channel scales
+def g16_row_bytes(D: int) -> int:
+    """Bytes of one entry in the 16-channel layout: D/2 codes, then D/16 scales."""
+    return D // 2 + D // 16
+
+
+def fp4_kv_pack_g16(kv: torch.Tensor, rows: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """kv float32 [B][N][D] -> rows uint8 [B][N][D/2 + D/16]."""
+    _want(kv, torch.float32, "kv", 3)
+    B, N, D = kv.shape
+    if rows is None:
+        rows = torch.empty((B, N, g16_row_bytes(D)), dtype=torch.uint8, device=kv.device)
+    _check(load().fp4_kv_pack_g16(_p(kv), B, N, D, _p(rows), _stream(kv.device)),
+           "fp4_kv_pack_g16")
+    return rows
+
+
+def fp4_kv_unpack_g16(rows: torch.Tensor, D: int) -> torch.Tensor:
+    _want(rows, torch.uint8, "rows", 3)
+    B, N, rb = rows.shape
+    if rb != g16_row_bytes(D):
+        raise ValueError("rows of %d bytes do not hold D=%d" % (rb, D))
+    out = torch.empty((B, N, D), dtype=torch.float32, device=rows.device)
+    _check(load().fp4_kv_unpack_g16(_p(rows), B, N, D, _p(out), _stream(rows.device)),
+           "fp4_kv_unpack_g16")
+    return out
+
+
+def fp4_kv_append_g16(rows: torch.Tensor, kv_new: torch.Tensor, pos: torch.Tensor) -> torch.Tensor:
+    """Quantise kv_new float32 [B][T][D] into rows[b][pos[b][t]] in place."""
+    _want(rows, torch.uint8, "rows", 3)
+    _want(kv_new, torch.float32, "kv_new", 3)
+    _want(pos, torch.int32, "pos", 2)
+    B, T, D = kv_new.shape
+    N = rows.shape[1]
+    _check(load().fp4_kv_append_g16(_p(kv_new), _p(pos), B, T, N, D, _p(rows),
+                                    _stream(rows.device)), "fp4_kv_append_g16")
+    return rows
 
 
 # ------------------------------------------------------------------- indexer
@@ -205,6 +251,32 @@ def csa2_sparse_attn(q: torch.Tensor, kv_packed: torch.Tensor, kv_scale: torch.T
                               float(softmax_scale), _p(out), _p(lse if want_lse else None),
                               _p(workspace) if need else None, need, _stream(q.device)),
            "csa2_sparse_attn")
+    return out, (lse if want_lse else None)
+
+
+def csa2_sparse_attn_g16(q: torch.Tensor, kv_rows: torch.Tensor, topk_idx: torch.Tensor,
+                         softmax_scale: float, want_lse: bool = True,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None):
+    """csa2_sparse_attn over a cache in the 16-channel layout (fp4_kv_pack_g16)."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want(kv_rows, torch.uint8, "kv_rows", 3)
+    _want(topk_idx, torch.int32, "topk_idx", 3)
+    B, Tq, Hq, D = q.shape
+    N = kv_rows.shape[1]
+    K = topk_idx.shape[-1]
+    L = load()
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=q.device)
+    need = L.csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(L.csa2_sparse_attn_g16(_p(q), _p(kv_rows), _p(topk_idx), B, Tq, Hq, D, N, K,
+                                  float(softmax_scale), _p(out), _p(lse if want_lse else None),
+                                  _p(workspace) if need else None, need, _stream(q.device)),
+           "csa2_sparse_attn_g16")
     return out, (lse if want_lse else None)
 
 

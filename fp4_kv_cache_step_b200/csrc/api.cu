@@ -87,6 +87,15 @@ csa2_status check_kv(const void* kv_packed, const void* kv_scale, int B, int N, 
   return CSA2_OK;
 }
 
+// The 16-channel layout: rows of D/2 + D/16 bytes; D % 128 == 0 keeps every
+// row 8-byte aligned (the kernels store a group's codes as one 8-byte word).
+csa2_status check_kv_g16(const void* kv_rows, int B, int N, int D) {
+  CHECK_PTR(kv_rows);
+  CHECK_ARG(B >= 0 && N >= 0, "B=%d and N=%d must be >= 0", B, N);
+  CHECK_ARG(D > 0 && D % 128 == 0, "D=%d must be a positive multiple of 128", D);
+  return CSA2_OK;
+}
+
 csa2_status check_score_args(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
                              int B, int Tq, int N, int Hi, int Di, const int32_t* nvalid,
                              const int32_t* cand, int C) {
@@ -110,6 +119,26 @@ csa2_status check_attn_args(const uint16_t* q, const uint8_t* kv_packed, const u
                             const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N, int K,
                             const uint16_t* out, const float* lse) {
   csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
+  if (s != CSA2_OK) return s;
+  CHECK_PTR(q);
+  CHECK_PTR(topk_idx);
+  CHECK_PTR(out);
+  if (lse) CHECK_ARG(((uintptr_t)lse & 3u) == 0, "lse must be 4-byte aligned");
+  CHECK_ARG(Tq >= 0, "Tq=%d must be >= 0", Tq);
+  CHECK_ARG(Hq >= 1 && Hq <= 65535, "Hq=%d must be in [1, 65535]", Hq);
+  CHECK_ARG(K >= 1, "K=%d must be >= 1", K);
+  if (D != csa2::kHeadDim)
+    return fail(CSA2_ERR_UNSUPPORTED, "attention is built for D=512 only (got D=%d)", D);
+  return CSA2_OK;
+}
+
+// Attention over the 16-channel layout (kv_rows) or the block layout.
+csa2_status check_attn_any(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                           const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N, int K,
+                           const uint16_t* out, const float* lse) {
+  if (kv_scale != nullptr)
+    return check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
+  csa2_status s = check_kv_g16(kv_packed, B, N, D);
   if (s != CSA2_OK) return s;
   CHECK_PTR(q);
   CHECK_PTR(topk_idx);
@@ -167,6 +196,44 @@ csa2_status fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale, int
   if (s != CSA2_OK) return s;
   cudaError_t e = csa2::launch_fp4_unpack(kv_packed, kv_scale, B, N, D, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack launch");
+  return ok();
+}
+
+csa2_status fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8_t* kv_rows,
+                            csa2_stream_t stream) {
+  CHECK_PTR(kv);
+  csa2_status s = check_kv_g16(kv_rows, B, N, D);
+  if (s != CSA2_OK) return s;
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "fp4_kv_pack_g16");
+  e = csa2::launch_fp4_pack_g16(kv, nullptr, B, N, N, D, kv_rows, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_pack_g16 launch");
+  return ok();
+}
+
+csa2_status fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, float* out,
+                              csa2_stream_t stream) {
+  CHECK_PTR(out);
+  csa2_status s = check_kv_g16(kv_rows, B, N, D);
+  if (s != CSA2_OK) return s;
+  cudaError_t e = csa2::launch_fp4_unpack_g16(kv_rows, B, N, D, out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack_g16 launch");
+  return ok();
+}
+
+csa2_status fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, int T, int N, int D,
+                              uint8_t* kv_rows, csa2_stream_t stream) {
+  CHECK_PTR(kv_new);
+  CHECK_PTR(pos);
+  CHECK_ARG(T >= 0, "T=%d must be >= 0", T);
+  csa2_status s = check_kv_g16(kv_rows, B, N, D);
+  if (s != CSA2_OK) return s;
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "fp4_kv_append_g16");
+  e = csa2::launch_fp4_pack_g16(kv_new, pos, B, T, N, D, kv_rows, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_append_g16 launch");
   return ok();
 }
 
@@ -232,6 +299,26 @@ csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const 
   return ok();
 }
 
+csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows,
+                                 const int32_t* topk_idx, int B, int Tq, int Hq, int D, int N,
+                                 int K, float softmax_scale, uint16_t* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, csa2_stream_t stream) {
+  csa2_status s = check_attn_any(q, kv_rows, nullptr, topk_idx, B, Tq, Hq, D, N, K, out, lse);
+  if (s != CSA2_OK) return s;
+  const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn_g16 needs %zu workspace bytes (got %zu)",
+                need, workspace_bytes);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_sparse_attn_g16");
+  // a NULL block-scale array selects the 16-channel layout
+  e = csa2::launch_sparse_attn(q, kv_rows, nullptr, topk_idx, B, Tq, Hq, N, K, softmax_scale, out,
+                               lse, workspace, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_sparse_attn_g16 launch");
+  return ok();
+}
+
 size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* a, csa2_mode mode,
                                        const csa2_shared_state* st) {
   if (!a || !st) return 0;
@@ -244,8 +331,9 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
   CHECK_ARG(a != nullptr && st != nullptr, "args and shared state must be non-null");
   CHECK_ARG(mode == CSA2_MODE_FULL || mode == CSA2_MODE_REINDEX || mode == CSA2_MODE_REUSE,
             "unknown mode %d", (int)mode);
-  csa2_status s = check_attn_args(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq,
-                                  a->Hq, a->D, a->N, a->K, a->out, a->lse);
+  // st->kv_scale NULL: st->kv_packed holds the 16-channel layout
+  csa2_status s = check_attn_any(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq,
+                                 a->Hq, a->D, a->N, a->K, a->out, a->lse);
   if (s != CSA2_OK) return s;
   const bool pooled = mode == CSA2_MODE_REINDEX && a->use_pool;
   const bool emit = mode == CSA2_MODE_FULL && a->emit_pool;

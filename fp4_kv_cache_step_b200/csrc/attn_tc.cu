@@ -162,8 +162,8 @@ __device__ __forceinline__ uint4 dq8(uint32_t codes, uint32_t s_lo, uint32_t s_h
 
 struct AttnParams {
   const uint16_t* q;
-  const uint8_t* kv_packed;
-  const uint8_t* kv_scale;
+  const uint8_t* kv_packed;     // codes [B][N][D/2]; or rows [B][N][D/2 + D/16] (16-channel scales)
+  const uint8_t* kv_scale;      // block scales [B][N/64][D]; unused for the 16-channel layout
   const int32_t* topk;
   int Tq, Hq, N, K, split_len, nsplit, nhb;
   float softmax_scale;
@@ -197,6 +197,10 @@ struct Raw {
   uint4 s[2];
 };
 
+// kG16: the cache is in the pages' own layout, one E4M3 scale per 16 channels
+// stored after the entry's codes (288 bytes per entry), instead of one scale
+// per channel per 64-entry block in a separate array.
+template <bool kG16>
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -250,8 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     // 8w + 2r + j, so each load of a warp covers whole 128-byte lines of two
     // rows (one line of codes or two of scales per row) instead of 32 rows.
     const int u = lane & 15, half = lane >> 4;
-    const uint8_t* pk_b = p.kv_packed + (size_t)b * p.N * (kD / 2);
-    const uint8_t* sc_b = p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
+    constexpr size_t kRowBytes = kG16 ? kD / 2 + kD / 16 : kD / 2;   // bytes of an entry's row
+    const uint8_t* pk_b = p.kv_packed + (size_t)b * p.N * kRowBytes;
+    const uint8_t* sc_b = kG16 ? nullptr : p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
     const int32_t* topk_row = p.topk + row * p.K;
 
     // lanes 0-7: index of entry 8w + lane of tile t, as loaded (checked later:
@@ -268,13 +273,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       return id;
     };
     // L2 prefetch of the warp's 8 rows: lane 4 j + q, q = 0, 1, half of the
-    // packed row of entry j; q = 2, 3, half of its scale row
+    // packed row of entry j; q = 2, 3, half of its scale row. A 288-byte row
+    // of the 16-channel layout starts 32-byte aligned, so lines q = 0, 1, 2
+    // cover it.
     auto prefetch_rows = [&](int ids) {
       const int id = __shfl_sync(0xffffffffu, ids, lane >> 2);
       if (id >= 0) {
         const int q = lane & 3;
-        if (q < 2) {
-          const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + q * 128;
+        if (kG16) {
+          if (q < 3) {
+            const uint8_t* pr = pk_b + (size_t)id * kRowBytes + q * 128;
+            asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(pr));
+          }
+        } else if (q < 2) {
+          const uint8_t* pr = pk_b + (size_t)id * kRowBytes + q * 128;
           asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(pr));
         } else {
           const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + (q - 2) * 256;
@@ -288,12 +300,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       for (int rr = 0; rr < 4; ++rr) {
         const int id = __shfl_sync(0xffffffffu, ids, 2 * rr + half);
         if (id >= 0) {
-          const uint8_t* pr = pk_b + (size_t)id * (kD / 2) + 8 * u;
-          const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + 16 * u;
+          const uint8_t* pr = pk_b + (size_t)id * kRowBytes + 8 * u;
           r[rr].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
           r[rr].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
-          r[rr].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
-          r[rr].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
+          if (kG16) {
+            // dims 16u .. 16u+15 are group u, dims 256+16u .. group 16+u: one
+            // scale byte each, repeated for the eight dims of a dequantised chunk
+            const uint8_t* sr = pk_b + (size_t)id * kRowBytes + kD / 2 + u;
+            const uint32_t s0 = 0x01010101u * __ldg(sr), s1 = 0x01010101u * __ldg(sr + 16);
+            r[rr].s[0] = make_uint4(s0, s0, s0, s0);
+            r[rr].s[1] = make_uint4(s1, s1, s1, s1);
+          } else {
+            const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + 16 * u;
+            r[rr].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
+            r[rr].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
+          }
         } else {
           r[rr].c[0] = r[rr].c[1] = make_uint2(0, 0);
           r[rr].s[0] = r[rr].s[1] = make_uint4(0, 0, 0, 0);
@@ -793,8 +814,10 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
   p.ws_ml = ws_ml;
   p.err = err;
   p.cluster_merge = 0;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // no block-scale array: rows of the 16-channel layout
+  void (*kernel)(AttnParams) =
+      kv_scale == nullptr ? sparse_attn_tc_kernel<true> : sparse_attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(rows, nhb, nsplit);
@@ -815,9 +838,9 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, sparse_attn_tc_kernel, &cfg) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg) == cudaSuccess &&
         nclusters > 0) {
-      e = launch_pdl(sparse_attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream,
+      e = launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream,
                      dim3(1, 1, (unsigned)nsplit), p);
       if (e == cudaSuccess) {
         *merged = true;
@@ -827,7 +850,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
     (void)cudaGetLastError();   // fall back to partials in the workspace
     p.cluster_merge = 0;
   }
-  return launch_pdl(sparse_attn_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, dim3(1), p);
+  return launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream, dim3(1), p);
 }
 
 }  // namespace csa2

@@ -52,6 +52,12 @@ cudaError_t launch_fp4_pack(const float* kv, int B, int N, int D, uint8_t* packe
                             uint8_t* scale, int* err, cudaStream_t stream);
 cudaError_t launch_fp4_unpack(const uint8_t* packed, const uint8_t* scale, int B, int N, int D,
                               float* out, cudaStream_t stream);
+// The 16-channel layout: rows [B][N][D/2 + D/16]. Entry t of row b of kv
+// ([B][T][D]) is quantised into cache row pos[b][t] (pos NULL: row t, T = N).
+cudaError_t launch_fp4_pack_g16(const float* kv, const int32_t* pos, int B, int T, int N, int D,
+                                uint8_t* rows, int* err, cudaStream_t stream);
+cudaError_t launch_fp4_unpack_g16(const uint8_t* rows, int B, int N, int D, float* out,
+                                  cudaStream_t stream);
 
 // Indexer scores; see csa2_index_score for the contract.
 cudaError_t launch_index_score(const uint8_t* idx_q, const float* idx_w, const uint8_t* idx_k,
@@ -70,7 +76,9 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
                         int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
                         int* err, cudaStream_t stream);
 
-// Sparse attention; see csa2_sparse_attn.
+// Sparse attention; see csa2_sparse_attn. With kv_scale NULL, kv_packed holds
+// the 16-channel layout (csa2_sparse_attn_g16): per entry D/2 code bytes then
+// D/16 E4M3 scale bytes.
 size_t sparse_attn_workspace_bytes(int B, int Tq, int Hq, int K);
 cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,

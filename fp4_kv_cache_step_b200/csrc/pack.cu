@@ -8,6 +8,13 @@
 // blockmax / 6; codes are the nearest E2M1 grid point with ties to the even
 // code. Both kernels are HBM-bound streaming kernels: 8 B read + 0.5 B
 // (+ 1/64 B of scale) written per value for the pack, the reverse for unpack.
+//
+// The same section and the interpretation's 3.5 give the production layout:
+// one E4M3 scale per 16 channels of an entry, with no second-level scale. The
+// *_g16 kernels store it as one row per entry, its D/2 code bytes followed by
+// its D/16 scale bytes (288 bytes at D = 512); a group's scale follows the same
+// rule (nearest E4M3 of max|x| / 6). Each row depends on its own entry alone,
+// so appending an entry writes its row and nothing else.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -130,7 +137,110 @@ __global__ void fp4_unpack_kernel(const uint8_t* __restrict__ packed,
   }
 }
 
+// One thread per 16-channel group of one source entry; the entry is written to
+// cache row pos[b][t] (pos NULL: row t).
+__global__ void fp4_pack_g16_kernel(const float* __restrict__ kv, const int32_t* __restrict__ pos,
+                                    int B, int T, int N, int D, uint8_t* __restrict__ rows,
+                                    int* err) {
+  const int groups = D / 16;
+  const size_t rb = (size_t)D / 2 + groups;
+  const size_t total = (size_t)B * T * groups;
+  for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total;
+       g += (size_t)gridDim.x * blockDim.x) {
+    const size_t src = g / groups;            // b * T + t
+    const int grp = (int)(g % groups);
+    const int b = (int)(src / T);
+    int n = (int)(src % T);
+    if (pos != nullptr) {
+      n = __ldg(pos + src);
+      if (n < 0 || n >= N) {
+        record_error(err, CSA2_ERR_DEVICE_INDEX);
+        continue;
+      }
+    }
+    const float4* x4 = reinterpret_cast<const float4*>(kv + src * D + grp * 16);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 f = __ldg(x4 + i);
+      v[4 * i] = f.x;
+      v[4 * i + 1] = f.y;
+      v[4 * i + 2] = f.z;
+      v[4 * i + 3] = f.w;
+    }
+    float amax = 0.0f;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      bad |= !isfinite(v[i]);
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+    if (bad) record_error(err, CSA2_ERR_NONFINITE);
+    // IEEE division then RNE to E4M3 (saturating), as in the block layout
+    const __nv_fp8_storage_t sc = __nv_cvt_float_to_fp8(amax / 6.0f, __NV_SATFINITE, __NV_E4M3);
+    const float s = __low2float(e4m3x2_to_half2((uint16_t)sc));
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i >> 3] |= e2m1_code(v[i], s) << (4 * (i & 7));
+    uint8_t* dst = rows + ((size_t)b * N + n) * rb;
+    *reinterpret_cast<uint2*>(dst + grp * 8) = make_uint2(w[0], w[1]);
+    dst[D / 2 + grp] = (uint8_t)sc;
+  }
+}
+
+// One thread per 16-channel group of one entry: exact values.
+__global__ void fp4_unpack_g16_kernel(const uint8_t* __restrict__ rows, int B, int N, int D,
+                                      float* __restrict__ out) {
+  const int groups = D / 16;
+  const size_t rb = (size_t)D / 2 + groups;
+  const size_t total = (size_t)B * N * groups;
+  for (size_t g = blockIdx.x * (size_t)blockDim.x + threadIdx.x; g < total;
+       g += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = g / groups;
+    const int grp = (int)(g % groups);
+    const uint8_t* src = rows + row * rb;
+    const uint2 c = *reinterpret_cast<const uint2*>(src + grp * 8);
+    const uint8_t sc = src[D / 2 + grp];
+    const __half2 s2 = e4m3x2_to_half2((uint16_t)(sc | (sc << 8)));
+    const uint32_t cw[2] = {c.x, c.y};
+    float res[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 f = __half22float2(
+          __hmul2(e2m1x2_to_half2((uint8_t)(cw[i >> 3] >> (4 * (i & 7)))), s2));   // exact
+      res[i] = f.x;
+      res[i + 1] = f.y;
+    }
+    float4* o = reinterpret_cast<float4*>(out + row * D + grp * 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = make_float4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+  }
+}
+
+int grid_for(size_t total, int threads) {
+  size_t blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  return (int)blocks;
+}
+
 }  // namespace
+
+cudaError_t launch_fp4_pack_g16(const float* kv, const int32_t* pos, int B, int T, int N, int D,
+                                uint8_t* rows, int* err, cudaStream_t stream) {
+  const size_t total = (size_t)B * T * (D / 16);
+  if (total == 0) return cudaSuccess;
+  fp4_pack_g16_kernel<<<grid_for(total, 256), 256, 0, stream>>>(kv, pos, B, T, N, D, rows, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp4_unpack_g16(const uint8_t* rows, int B, int N, int D, float* out,
+                                  cudaStream_t stream) {
+  const size_t total = (size_t)B * N * (D / 16);
+  if (total == 0) return cudaSuccess;
+  fp4_unpack_g16_kernel<<<grid_for(total, 256), 256, 0, stream>>>(rows, B, N, D, out);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fp4_pack(const float* kv, int B, int N, int D, uint8_t* packed,
                             uint8_t* scale, int* err, cudaStream_t stream) {

@@ -31,8 +31,10 @@
  *    16-bit patterns (uint16_t), E4M3 values as bytes.
  *  - Packed FP4: byte c/2 of an entry holds channel c, low nibble = even c.
  *    Scales: one E4M3 byte per channel per 64-entry block,
- *    kv_scale[b][n/64][c] (this block-scale layout is the one the benchmark
- *    configurations state; the pages' own 16-channel grouping is not built).
+ *    kv_scale[b][n/64][c] (the block-scale layout the benchmark
+ *    configurations state). The pages' own layout, one E4M3 scale per 16
+ *    channels of an entry, has its own calls (*_g16): an entry is one row of
+ *    D/2 code bytes followed by D/16 scale bytes, kv_rows[b][n][D/2 + D/16].
  *  - Pointers must be 16-byte aligned; D must be 512 for attention; N must be a
  *    multiple of 64.
  */
@@ -100,6 +102,46 @@ CSA2_API csa2_status fp4_kv_pack(const float* kv, int B, int N, int D,
  *   out        float   [B][N][D]      output (every value is exact in fp32) */
 CSA2_API csa2_status fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale,
                           int B, int N, int D, float* out, csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fp4_kv_pack_g16 -- quantise the main KV cache in the pages' own layout:
+ * E2M1 values with one E4M3 scale per 16 channels of an entry and no
+ * second-level global scale ([N] "FP4 Main KV Cache To Halve Storage Again";
+ * [M] 3.5). Where the scale bytes sit and how a scale is chosen is not stated;
+ * this library stores each entry as one row, its D/2 code bytes then its D/16
+ * scale bytes (288 bytes at D = 512), and takes the block layout's rule per
+ * group: scale = nearest-even E4M3 of max|x| / 6 (saturating at 448), codes as
+ * in fp4_kv_pack.
+ *   kv       float [B][N][D]              input, finite
+ *   kv_rows  uint8 [B][N][D/2 + D/16]     output; group g's scale is byte
+ *                                         D/2 + g of the row (channels
+ *                                         16g .. 16g + 15)
+ * Requires D % 128 == 0 (every row 8-byte aligned); N is free. A NaN or
+ * infinity records CSA2_ERR_NONFINITE on the device (the row is still written).
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8_t* kv_rows,
+                                     csa2_stream_t stream);
+
+/* fp4_kv_unpack_g16 -- exact dequantisation of the 16-channel layout:
+ * out[b][n][c] = e2m1(code) * e4m3(scale of group c / 16).
+ *   out      float [B][N][D]              output */
+CSA2_API csa2_status fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, float* out,
+                                       csa2_stream_t stream);
+
+/* fp4_kv_append_g16 -- quantise new entries into an existing cache of the
+ * 16-channel layout (entries are quantised after the rotary embedding,
+ * [N] "FP4 Main KV Cache To Halve Storage Again"; [M] 3.5, so the caller
+ * passes post-RoPE values). Entry t of row b goes to cache row pos[b][t];
+ * every other row is left as it is, since each row carries its own scales.
+ *   kv_new   float [B][T][D]              input, finite
+ *   pos      int32 [B][T]                 destination rows in [0, N); a
+ *                                         position outside it is skipped and
+ *                                         CSA2_ERR_DEVICE_INDEX recorded; the
+ *                                         positions of one b must differ
+ *   kv_rows  uint8 [B][N][D/2 + D/16]     updated in place
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, int T,
+                                       int N, int D, uint8_t* kv_rows, csa2_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * csa2_index_score -- indexer scores ([N] "Compressed Sparse Attention 2 Or
@@ -171,6 +213,18 @@ CSA2_API csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packe
                              float softmax_scale, uint16_t* out, float* lse,
                              void* workspace, size_t workspace_bytes, csa2_stream_t stream);
 
+/* csa2_sparse_attn_g16 -- csa2_sparse_attn over a cache in the 16-channel
+ * layout (fp4_kv_pack_g16): the same computation, with v_k dequantised from
+ * row idx_k's codes and its own group scales. Same arguments otherwise, the
+ * same workspace (csa2_sparse_attn_workspace_bytes), D == 512 (288-byte rows),
+ * any N >= 0.
+ *   kv_rows  uint8 [B][N][D/2 + D/16] */
+CSA2_API csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows,
+                                          const int32_t* topk_idx, int B, int Tq, int Hq, int D,
+                                          int N, int K, float softmax_scale, uint16_t* out,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          csa2_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * csa2_sparse_attn_noalloc -- csa2_sparse_attn without a caller workspace.
  * (An interface addition of this library; the pages describe no such call.)
@@ -214,8 +268,10 @@ CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* 
  *   REUSE   : attention over st->topk_idx as it stands
  * ------------------------------------------------------------------------ */
 typedef struct {
-  const uint8_t* kv_packed;   /* [B][N][D/2] */
-  const uint8_t* kv_scale;    /* [B][N/64][D] */
+  const uint8_t* kv_packed;   /* [B][N][D/2]; with kv_scale NULL, the rows
+                                 [B][N][D/2 + D/16] of the 16-channel layout
+                                 (fp4_kv_pack_g16) */
+  const uint8_t* kv_scale;    /* [B][N/64][D]; NULL selects the 16-channel layout */
   const uint8_t* idx_k;       /* [B][N][Di] E4M3; may be NULL when only REUSE runs */
   int32_t* topk_idx;          /* [B][Tq][K]: written by FULL/REINDEX, read by all */
   int32_t* cand_idx;          /* [B][Tq][C]: written by FULL (emit_pool), read by REINDEX (use_pool) */

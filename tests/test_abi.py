@@ -125,3 +125,21 @@ def test_workspace_query_for_layer_modes(lib):
     assert 4 * 8192 * 4 <= b_pool < b_full
     b_reuse = lib.csa2_layer_step_workspace_bytes(ctypes.byref(pooled), 2, ctypes.byref(sh))
     assert b_reuse < b_pool
+
+
+def test_g16_layout_arguments_are_checked(lib):
+    P = ctypes.c_void_p
+    a = P(256)
+    # rows of the 16-channel layout need D % 128 == 0 (8-byte aligned rows)
+    assert _status(lib.fp4_kv_pack_g16(a, 1, 64, 96, a, None)) == "INVALID_ARG"
+    assert _status(lib.fp4_kv_pack_g16(a, 1, 64, 512, None, None)) == "INVALID_ARG"
+    assert _status(lib.fp4_kv_unpack_g16(a, 1, 64, 512, P(8), None)) == "INVALID_ARG"
+    assert _status(lib.fp4_kv_append_g16(a, a, 1, -1, 64, 512, a, None)) == "INVALID_ARG"
+    assert _status(lib.fp4_kv_append_g16(a, None, 1, 2, 64, 512, a, None)) == "INVALID_ARG"
+    # attention over the layout is built for D = 512, like the block layout
+    rc = lib.csa2_sparse_attn_g16(a, a, a, 1, 1, 16, 256, 64, 8, ctypes.c_float(1.0), a, None,
+                                  None, 0, None)
+    assert _status(rc) == "UNSUPPORTED"
+    rc = lib.csa2_sparse_attn_g16(a, a, a, 2, 1, 64, 512, 100, 2048, ctypes.c_float(1.0), a, None,
+                                  None, 0, None)
+    assert _status(rc) == "WORKSPACE"
