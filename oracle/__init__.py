@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.or_fp4_kv_unpack_g16.argtypes = [P, I, I, I, P]
         L.or_fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P]
         L.or_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, D, P, P]
+        L.or_block_pool.argtypes = [P, I, I, P, I, I, P]
         L.or_index_score.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
         L.or_topk.argtypes = [P, I, I, P, P, I, P]
         L.or_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, P]
@@ -73,7 +74,8 @@ def lib() -> ctypes.CDLL:
                                     P, P, P, P]
         for f in (L.or_fp4_kv_pack, L.or_fp4_kv_unpack, L.or_index_score, L.or_topk,
                   L.or_sparse_attn, L.or_dense_attn, L.or_layer_step, L.or_fp4_kv_pack_g16,
-                  L.or_fp4_kv_unpack_g16, L.or_fp4_kv_append_g16, L.or_sparse_attn_g16):
+                  L.or_fp4_kv_unpack_g16, L.or_fp4_kv_append_g16, L.or_sparse_attn_g16,
+                  L.or_block_pool):
             f.restype = I
         _lib = L
     return _lib
@@ -227,6 +229,21 @@ def topk(scores, K, nvalid=None, cand=None) -> np.ndarray:
     cd = None if cand is None else _c(cand, np.int32)
     out = np.zeros(lead + (K,), np.int32)
     _check(lib().or_topk(_ptr(scores), rows, ld, _ptr(nv), _ptr(cd), K, _ptr(out)), "or_topk")
+    return out
+
+
+def block_pool(scores, nvalid, block: int, nblocks: int) -> np.ndarray:
+    """scores [..., ld] (float64), nvalid [...] -> int32 [..., nblocks*block]:
+    the valid positions of the best `nblocks` blocks of `block` positions
+    (block score = max over its valid positions), ascending, -1 padded."""
+    scores = _c(scores, np.float64)
+    lead = scores.shape[:-1]
+    ld = scores.shape[-1]
+    rows = int(np.prod(lead)) if lead else 1
+    nv = _c(nvalid, np.int32)
+    out = np.zeros(lead + (nblocks * block,), np.int32)
+    _check(lib().or_block_pool(_ptr(scores), rows, ld, _ptr(nv), int(block), int(nblocks),
+                               _ptr(out)), "or_block_pool")
     return out
 
 

@@ -362,6 +362,56 @@ int or_topk(const double* scores, int rows, int ld,
     return rc;
 }
 
+/* Blockwise candidate pool of the hierarchical indexer ("Detailed Notes On
+ * DeepSeek V4 Point 1 Flash In Simple Words", "Hierarchical Sparse Indexer In
+ * Simple Terms"; mengman.github.io 3.4): the first FULL layer groups positions
+ * into blocks of `block`, scores each block by the maximum score of its valid
+ * positions, keeps the best `nblocks` blocks (ranked like entries: block score
+ * descending, block index ascending) and hands their positions to the later
+ * REINDEX layers. Output per row: the kept blocks' valid positions ascending,
+ * padded with -1 to nblocks * block. */
+int or_block_pool(const double* scores, int rows, int ld, const int32_t* nvalid,
+                  int block, int nblocks, int32_t* cand) {
+    if (!scores || !nvalid || !cand || rows < 0 || ld < 0 || block <= 0 || nblocks <= 0)
+        return OR_BAD_ARG;
+    const int nbmax = (ld + block - 1) / block;
+    const size_t C = (size_t)nblocks * block;
+    double* bscore = (double*)malloc(sizeof(double) * (size_t)(nbmax > 0 ? nbmax : 1));
+    int32_t* kept = (int32_t*)malloc(sizeof(int32_t) * (size_t)nblocks);
+    if (!bscore || !kept) { free(bscore); free(kept); return OR_BAD_ARG; }
+    int rc = OR_OK;
+    for (int r = 0; r < rows && rc == OR_OK; ++r) {
+        const int nv = nvalid[r];
+        if (nv < 0 || nv > ld) { rc = OR_BAD_ARG; break; }
+        const int nb = (nv + block - 1) / block;          /* blocks with a valid position */
+        for (int bk = 0; bk < nb; ++bk) {
+            double m = -INFINITY;
+            for (int j = bk * block; j < (bk + 1) * block && j < nv; ++j) {
+                double x = scores[(size_t)r * ld + j];
+                if (isnan(x)) { rc = OR_NONFINITE; break; }
+                if (x > m) m = x;
+            }
+            bscore[bk] = m;
+        }
+        if (rc != OR_OK) break;
+        /* the best blocks, by the entries' own ranking rule */
+        rc = or_topk(bscore, 1, nb > 0 ? nb : 0, &nb, NULL, nblocks, kept);
+        if (rc != OR_OK) break;
+        size_t n = 0;
+        for (int i = 0; i < nblocks; ++i) {
+            if (kept[i] < 0) continue;
+            for (int t = 0; t < block; ++t) {
+                int j = kept[i] * block + t;
+                if (j < nv) cand[(size_t)r * C + n++] = j;
+            }
+        }
+        while (n < C) cand[(size_t)r * C + n++] = -1;
+    }
+    free(bscore);
+    free(kept);
+    return rc;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Sparse softmax attention over the selected rows; K doubles as V.          */
 /* ------------------------------------------------------------------------ */

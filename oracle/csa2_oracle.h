@@ -93,6 +93,13 @@ int or_topk(const double* scores, int rows, int ld,
             const int32_t* nvalid, const int32_t* cand,
             int K, int32_t* topk);
 
+/* Blockwise candidate pool: blocks of `block` positions scored by the maximum
+ * over their valid positions (j < nvalid[r]); the top `nblocks` blocks by
+ * (block score descending, block index ascending) are kept and their valid
+ * positions written ascending to cand[r][0 .. nblocks*block), -1 padded. */
+int or_block_pool(const double* scores, int rows, int ld, const int32_t* nvalid,
+                  int block, int nblocks, int32_t* cand);
+
 int or_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
                    const int32_t* topk, int B, int Tq, int Hq, int D, int N, int K,
                    double softmax_scale, double* out, double* lse);
