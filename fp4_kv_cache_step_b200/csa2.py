@@ -49,7 +49,8 @@ EXPORTS = ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk",
            "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn",
            "csa2_layer_step_workspace_bytes", "csa2_layer_step", "csa2_check_device_errors",
            "csa2_last_error", "csa2_sparse_attn_noalloc", "fp4_kv_pack_g16", "fp4_kv_unpack_g16",
-           "fp4_kv_append_g16", "csa2_sparse_attn_g16")
+           "fp4_kv_append_g16", "csa2_sparse_attn_g16", "csa2_block_pool_workspace_bytes",
+           "csa2_block_pool")
 
 _lib = None
 
@@ -76,6 +77,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp4_kv_unpack_g16.argtypes = [P, I, I, I, P, P]
     L.fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P, P]
     L.csa2_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
+    L.csa2_block_pool_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.csa2_block_pool_workspace_bytes.restype = Z
+    L.csa2_block_pool.argtypes = [P, I, P, I, I, I, I, P, P, Z, P]
     L.csa2_layer_step_workspace_bytes.argtypes = [ctypes.POINTER(LayerArgs), I,
                                                   ctypes.POINTER(SharedState)]
     L.csa2_layer_step_workspace_bytes.restype = Z
@@ -85,7 +89,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.csa2_last_error.restype = ctypes.c_char_p
     for f in ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk", "csa2_sparse_attn",
               "csa2_layer_step", "csa2_check_device_errors", "csa2_sparse_attn_noalloc",
-              "fp4_kv_pack_g16", "fp4_kv_unpack_g16", "fp4_kv_append_g16", "csa2_sparse_attn_g16"):
+              "fp4_kv_pack_g16", "fp4_kv_unpack_g16", "fp4_kv_append_g16", "csa2_sparse_attn_g16",
+              "csa2_block_pool"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -228,6 +233,25 @@ def csa2_topk(scores: torch.Tensor, K: int, nvalid: Optional[torch.Tensor] = Non
     return (out, cand_out) if Cout else out
 
 
+def csa2_block_pool(scores: torch.Tensor, nvalid: torch.Tensor, nblocks: int, block: int = 8,
+                    out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """scores float32 [B][Tq][ld] -> the blockwise pool int32 [B][Tq][nblocks * block]."""
+    _want(scores, torch.float32, "scores", 3)
+    _want(nvalid, torch.int32, "nvalid", 2)
+    B, Tq, ld = scores.shape
+    L = load()
+    if out is None:
+        out = torch.empty((B, Tq, nblocks * block), dtype=torch.int32, device=scores.device)
+    need = L.csa2_block_pool_workspace_bytes(B, Tq, ld, block, nblocks)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=scores.device)
+    _check(L.csa2_block_pool(_p(scores), ld, _p(nvalid), B, Tq, int(block), int(nblocks), _p(out),
+                             _p(workspace) if need else None, need, _stream(scores.device)),
+           "csa2_block_pool")
+    return out
+
+
 # ------------------------------------------------------------------- attention
 def csa2_sparse_attn(q: torch.Tensor, kv_packed: torch.Tensor, kv_scale: torch.Tensor,
                      topk_idx: torch.Tensor, softmax_scale: float, want_lse: bool = True,
@@ -319,12 +343,13 @@ class Csa2Shared:
 
 def layer_args(q, nvalid, out, K, softmax_scale, idx_q=None, idx_w=None, lse=None, N=None,
                emit_pool=False, use_pool=False) -> LayerArgs:
+    """emit_pool: False/0 none, True/1 the top-C entries, 2 the blockwise pool."""
     B, Tq, Hq, D = q.shape
     Hi = Di = 0
     if idx_q is not None:
         Hi, Di = idx_q.shape[2], idx_q.shape[3]
     return LayerArgs(B, Tq, int(N), D, Hq, Hi, Di, int(K), _p(nvalid), _p(q), _p(idx_q),
-                     _p(idx_w), float(softmax_scale), _p(out), _p(lse), int(bool(emit_pool)),
+                     _p(idx_w), float(softmax_scale), _p(out), _p(lse), int(emit_pool),
                      int(bool(use_pool)))
 
 

@@ -319,10 +319,48 @@ csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows,
   return ok();
 }
 
+size_t csa2_block_pool_workspace_bytes(int B, int Tq, int ld, int block, int nblocks) {
+  if (B <= 0 || Tq <= 0) return 0;
+  return round_up(csa2::block_pool_workspace_bytes(B * Tq, ld, block, nblocks));
+}
+
+csa2_status csa2_block_pool(const float* scores, int ld, const int32_t* nvalid, int B, int Tq,
+                            int block, int nblocks, int32_t* cand_out, void* workspace,
+                            size_t workspace_bytes, csa2_stream_t stream) {
+  CHECK_PTR(scores);
+  CHECK_PTR(nvalid);
+  CHECK_PTR(cand_out);
+  CHECK_ARG(B >= 0 && Tq >= 0, "B=%d and Tq=%d must be >= 0", B, Tq);
+  CHECK_ARG(ld >= 0 && ld <= (1 << 30), "ld=%d must be in [0, 2^30]", ld);
+  CHECK_ARG(block >= 1 && nblocks >= 1 && nblocks <= 65536,
+            "block=%d must be >= 1 and nblocks=%d in [1, 65536]", block, nblocks);
+  CHECK_ARG((long long)block * nblocks <= (1 << 30), "block x nblocks must be <= 2^30");
+  const size_t need = csa2_block_pool_workspace_bytes(B, Tq, ld, block, nblocks);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA2_ERR_WORKSPACE, "csa2_block_pool needs %zu workspace bytes (got %zu)", need,
+                workspace_bytes);
+  cudaError_t e;
+  int* err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "csa2_block_pool");
+  e = csa2::launch_block_pool(scores, ld, nvalid, B * Tq, block, nblocks, cand_out, workspace, err,
+                              (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_block_pool launch");
+  return ok();
+}
+
+// FULL with emit_pool == 2: the blockwise pool, blocks of 8, C / 8 of them
+constexpr int kPoolBlock = 8;
+
+static size_t layer_pool_bytes(const csa2_layer_args* a, csa2_mode mode,
+                               const csa2_shared_state* st) {
+  if (mode != CSA2_MODE_FULL || a->emit_pool != 2 || st->C < kPoolBlock) return 0;
+  return csa2_block_pool_workspace_bytes(a->B, a->Tq, a->N, kPoolBlock, st->C / kPoolBlock);
+}
+
 size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* a, csa2_mode mode,
                                        const csa2_shared_state* st) {
   if (!a || !st) return 0;
-  return layer_scores_bytes(a, mode, st) +
+  return layer_scores_bytes(a, mode, st) + layer_pool_bytes(a, mode, st) +
          csa2_sparse_attn_workspace_bytes(a->B, a->Tq, a->Hq, a->D, a->K);
 }
 
@@ -337,6 +375,9 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
   if (s != CSA2_OK) return s;
   const bool pooled = mode == CSA2_MODE_REINDEX && a->use_pool;
   const bool emit = mode == CSA2_MODE_FULL && a->emit_pool;
+  const bool emit_blocks = emit && a->emit_pool == 2;
+  CHECK_ARG(a->emit_pool >= 0 && a->emit_pool <= 2, "emit_pool=%d must be 0, 1 or 2",
+            a->emit_pool);
   if (mode != CSA2_MODE_REUSE) {
     s = check_score_args(a->idx_q, a->idx_w, st->idx_k, a->B, a->Tq, a->N, a->Hi, a->Di, a->nvalid,
                          pooled ? st->cand_idx : nullptr, st->C);
@@ -346,7 +387,11 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
       CHECK_PTR(st->cand_idx);
       CHECK_ARG(st->C >= 1 && st->C <= 65536, "pool size C=%d must be in [1, 65536]", st->C);
     }
-    if (emit) CHECK_ARG(st->C >= a->K, "pool size C=%d must be >= K=%d", st->C, a->K);
+    if (emit && !emit_blocks)
+      CHECK_ARG(st->C >= a->K, "pool size C=%d must be >= K=%d", st->C, a->K);
+    if (emit_blocks)
+      CHECK_ARG(st->C % kPoolBlock == 0 && st->C / kPoolBlock >= a->K,
+                "a blockwise pool needs C=%d a multiple of 8 with C/8 >= K=%d", st->C, a->K);
   }
   const size_t need = csa2_layer_step_workspace_bytes(a, mode, st);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
@@ -358,6 +403,7 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
   cudaStream_t cs = (cudaStream_t)stream;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   const size_t scores_bytes = layer_scores_bytes(a, mode, st);
+  const size_t pool_bytes = layer_pool_bytes(a, mode, st);
   if (mode != CSA2_MODE_REUSE) {
     float* scores = reinterpret_cast<float*>(ws);
     const int ld = pooled ? st->C : a->N;
@@ -365,14 +411,20 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
                                  a->nvalid, pooled ? st->cand_idx : nullptr, pooled ? st->C : 0,
                                  scores, err, cs);
     if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step score");
+    const bool emit_entries = emit && !emit_blocks;
     e = csa2::launch_topk(scores, ld, pooled ? nullptr : a->nvalid, pooled ? st->cand_idx : nullptr,
-                          a->B * a->Tq, a->K, st->topk_idx, emit ? st->C : 0,
-                          emit ? st->cand_idx : nullptr, err, cs);
+                          a->B * a->Tq, a->K, st->topk_idx, emit_entries ? st->C : 0,
+                          emit_entries ? st->cand_idx : nullptr, err, cs);
     if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step top-k");
+    if (emit_blocks) {
+      e = csa2::launch_block_pool(scores, a->N, a->nvalid, a->B * a->Tq, kPoolBlock,
+                                  st->C / kPoolBlock, st->cand_idx, ws + scores_bytes, err, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step block pool");
+    }
   }
   e = csa2::launch_sparse_attn(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq, a->Hq,
                                a->N, a->K, a->softmax_scale, a->out, a->lse,
-                               ws ? ws + scores_bytes : nullptr, err, cs);
+                               ws ? ws + scores_bytes + pool_bytes : nullptr, err, cs);
   if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step attention");
   return ok();
 }

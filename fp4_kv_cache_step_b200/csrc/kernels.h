@@ -76,6 +76,12 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
                         int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
                         int* err, cudaStream_t stream);
 
+// Blockwise candidate pool (pool.cu); see csa2_block_pool.
+size_t block_pool_workspace_bytes(int rows, int ld, int block, int nblocks);
+cudaError_t launch_block_pool(const float* scores, int ld, const int32_t* nvalid, int rows,
+                              int block, int nblocks, int32_t* cand, void* workspace, int* err,
+                              cudaStream_t stream);
+
 // Sparse attention; see csa2_sparse_attn. With kv_scale NULL, kv_packed holds
 // the 16-channel layout (csa2_sparse_attn_g16): per entry D/2 code bytes then
 // D/16 E4M3 scale bytes.

@@ -189,6 +189,29 @@ CSA2_API csa2_status csa2_topk(const float* scores, int ld, const int32_t* nvali
                       int Cout, int32_t* cand_out, csa2_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_block_pool -- the blockwise candidate pool of the hierarchical indexer
+ * ([N] "Hierarchical Sparse Indexer In Simple Terms"; [M] 3.4): the first FULL
+ * layer groups positions into blocks of `block` (8 in the model), scores each
+ * block by the largest score among its valid positions (j < nvalid), keeps the
+ * best `nblocks` blocks (2048 in the model: about 16384 candidates) ranked like
+ * entries (block score descending, lower block index first) and gives their
+ * valid positions to later REINDEX layers as the pool (csa2_index_score and
+ * csa2_topk with `cand`).
+ *   scores   float [B][Tq][ld]               from csa2_index_score (full scan)
+ *   nvalid   int32 [B][Tq]                   clamped to [0, ld]
+ *   cand_out int32 [B][Tq][nblocks * block]  ascending positions, -1 padded
+ *   workspace device scratch of csa2_block_pool_workspace_bytes() bytes
+ * Requires 1 <= nblocks <= 65536, block >= 1, block * nblocks <= 2^30. A NaN
+ * score records CSA2_ERR_NONFINITE.
+ * ------------------------------------------------------------------------ */
+CSA2_API size_t csa2_block_pool_workspace_bytes(int B, int Tq, int ld, int block, int nblocks);
+
+CSA2_API csa2_status csa2_block_pool(const float* scores, int ld, const int32_t* nvalid, int B,
+                                     int Tq, int block, int nblocks, int32_t* cand_out,
+                                     void* workspace, size_t workspace_bytes,
+                                     csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa2_sparse_attn -- gather + FP4 dequantisation + softmax attention over
  * the selected entries only ([N] CSA2 section and "FP4 Main KV Cache To Halve
  * Storage Again": values are dequantised back before attention). One shared
@@ -260,8 +283,11 @@ CSA2_API csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* 
  * device pointers that several layers pass to each other without copies: the
  * main KV and indexer keys built by a FULL layer, and the latest top-K indices
  * (and candidate pool) that REINDEX/REUSE layers consume.
- *   FULL    : score [0, nvalid) -> top-K into st->topk_idx (and the top-C pool
- *             into st->cand_idx when args->emit_pool and st->C > 0) -> attention
+ *   FULL    : score [0, nvalid) -> top-K into st->topk_idx (and, when
+ *             args->emit_pool and st->C > 0, a pool into st->cand_idx: the
+ *             top-C entries for emit_pool == 1, or the blockwise pool of
+ *             csa2_block_pool with blocks of 8 and C / 8 blocks for
+ *             emit_pool == 2) -> attention
  *   REINDEX : score [0, nvalid), or only st->cand_idx when args->use_pool,
  *             with this layer's own indexer query -> top-K into st->topk_idx
  *             -> attention
@@ -287,7 +313,8 @@ typedef struct {
   float softmax_scale;
   uint16_t* out;              /* [B][Tq][Hq][D] bf16 */
   float* lse;                 /* [B][Tq][Hq] or NULL */
-  int emit_pool;              /* FULL: also write the top-C pool into st->cand_idx */
+  int emit_pool;              /* FULL: 0 no pool; 1 the top-C entries; 2 the blockwise
+                                 pool (blocks of 8, C/8 blocks, C % 8 == 0) into st->cand_idx */
   int use_pool;               /* REINDEX: score only st->cand_idx */
 } csa2_layer_args;
 

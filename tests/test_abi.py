@@ -143,3 +143,25 @@ def test_g16_layout_arguments_are_checked(lib):
     rc = lib.csa2_sparse_attn_g16(a, a, a, 2, 1, 64, 512, 100, 2048, ctypes.c_float(1.0), a, None,
                                   None, 0, None)
     assert _status(rc) == "WORKSPACE"
+
+
+def test_block_pool_arguments_are_checked(lib):
+    P = ctypes.c_void_p
+    a = P(256)
+    assert _status(lib.csa2_block_pool(a, 100, a, 1, 1, 8, 0, a, a, 1 << 20, None)) == "INVALID_ARG"
+    assert _status(lib.csa2_block_pool(a, 100, a, 1, 1, 0, 4, a, a, 1 << 20, None)) == "INVALID_ARG"
+    assert _status(lib.csa2_block_pool(a, 100, None, 1, 1, 8, 4, a, a, 1 << 20, None)) == "INVALID_ARG"
+    need = lib.csa2_block_pool_workspace_bytes(2, 1, 262144, 8, 2048)
+    assert need >= 2 * (32768 * 4 + 2048 * 4)
+    assert _status(lib.csa2_block_pool(a, 262144, a, 2, 1, 8, 2048, a, a, need - 256, None)) == \
+        "WORKSPACE"
+
+
+def test_layer_step_blockwise_pool_needs_a_multiple_of_eight(lib):
+    sh = csa2.SharedState(256, 256, 256, 256, 256, 8190)
+    args = csa2.LayerArgs(1, 1, 4096, 512, 16, 4, 64, 256, 256, 256, 256, 256, 1.0, 256, None, 2, 0)
+    rc = lib.csa2_layer_step(ctypes.byref(args), 0, ctypes.byref(sh), None, 0, None)
+    assert _status(rc) == "INVALID_ARG" and b"multiple of 8" in lib.csa2_last_error()
+    args.emit_pool = 3
+    rc = lib.csa2_layer_step(ctypes.byref(args), 0, ctypes.byref(sh), None, 0, None)
+    assert _status(rc) == "INVALID_ARG"
