@@ -240,7 +240,12 @@ def run_ours(args):
 
     # ---- per-kernel timing: the same kernels through the individual calls
     nsplit_ws = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K)
-    kern = {"score": [], "topk": [], "attn": []}
+    kern = {"score": [], "topk": [], "attn": [], "block_pool": []}
+    # the hierarchical indexer's blockwise pool (2048 blocks of 8), as a FULL
+    # decoder layer emits it right after its top-K, from the same scores
+    pool_out = torch.empty((w.B, w.Tq, 2048 * 8), dtype=torch.int32, device=dev)
+    pool_ws = torch.empty(max(int(csa2.load().csa2_block_pool_workspace_bytes(
+        w.B, w.Tq, w.N, 8, 2048)), 256), dtype=torch.uint8, device=dev)
     scores = torch.empty((w.B, w.Tq, w.N), dtype=torch.float32, device=dev)
     ws = torch.empty(max(int(nsplit_ws), 256), dtype=torch.uint8, device=dev)
     out = torch.empty_like(dw.out[0])
@@ -253,6 +258,9 @@ def run_ours(args):
         evs[1].record(stream)
         csa2.csa2_topk(scores, w.K, nvalid=dw.nvalid, out=dw.topk)
         evs[2].record(stream)
+        e_pool = torch.cuda.Event(enable_timing=True)
+        csa2.csa2_block_pool(scores, dw.nvalid, 2048, 8, out=pool_out, workspace=pool_ws)
+        e_pool.record(stream)
         flush_l2(i)
         evs[3].record(stream)
         csa2.csa2_sparse_attn(dw.q[0], dw.kv_packed, dw.kv_scale, dw.topk, w.softmax_scale,
@@ -264,6 +272,7 @@ def run_ours(args):
             kern["score"].append(evs[0].elapsed_time(evs[1]))
             kern["topk"].append(evs[1].elapsed_time(evs[2]))
             kern["attn"].append(evs[3].elapsed_time(e4))
+            kern["block_pool"].append(evs[2].elapsed_time(e_pool))
     kern_us = {k: 1e3 * statistics.mean(v) for k, v in kern.items()}
 
     nvalid = wl.nvalid(w)
