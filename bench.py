@@ -495,6 +495,66 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_stack(args):
+    """One decode step of the model's own CSA2 layers (workloads.production_stack:
+    three encoder groups [FULL + 5 REUSE] over caches of T/2 entries, the
+    decoder's [FULL + 3 REUSE] + 4 x [REINDEX + 3 REUSE] over a cache of T
+    entries with the blockwise pool; top-512, indexer 32 x 128), timed with
+    device events over whole steps, L2 flushed between steps. One GPU."""
+    import torch
+
+    from fp4_kv_cache_step_b200 import csa2
+    from fp4_kv_cache_step_b200 import workloads as wl
+    from fp4_kv_cache_step_b200.runner import DeviceStack
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    csa2.load()
+    st = wl.production_stack(args.context, args.batch)
+    ds = DeviceStack(st, dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    for _ in range(args.warmup):
+        ds.step()
+    torch.cuda.synchronize()
+    csa2.check_device_errors()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            flush_rd.max()
+            ev[i][0].record(stream)
+            ds.step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    csa2.check_device_errors()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    ms_per_step = sum(ms) / len(ms)
+    nlayers = len(st.layers)
+    modes = [st.segments[s].modes[l] for s, l in st.layers]
+    launches = sum({"FULL": 3, "REINDEX": 3, "REUSE": 1}[m] for m in modes)
+    launches += 3                                      # the decoder FULL's blockwise pool
+    print(json.dumps({
+        "metric": "CSA2 stack decode steps/s (the model's 38 CSA2 layers)",
+        "value": 1e3 / ms_per_step, "unit": "stack-steps/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "production_stack", "context_tokens": args.context,
+                   "B": args.batch, "csa2_layers": nlayers, "swa_only_layers": st.swa_only,
+                   "encoder_entries": args.context // 2, "decoder_entries": args.context,
+                   "K": wl.PROD_K, "Hi": wl.PROD_HI, "Di": wl.PROD_DI, "Hq": wl.PROD_HQ,
+                   "pool": "%d blocks of %d" % (wl.PROD_POOL_BLOCKS, wl.PROD_POOL_BLOCK),
+                   "modes": {m: modes.count(m) for m in ("FULL", "REINDEX", "REUSE")},
+                   "l2": "flushed between timed steps"},
+        "per_layer_us": 1e3 * ms_per_step / nlayers,
+        "query_tokens_per_s": args.batch * 1e3 / ms_per_step,
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -507,10 +567,16 @@ def main():
     ap.add_argument("--attn-bound", default="tensor", choices=["tensor", "hbm"])
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if captured")
+    ap.add_argument("--stack", default=None, choices=["production"],
+                    help="time the model's 38 CSA2 layers (one GPU) instead of the headline step")
+    ap.add_argument("--context", type=int, default=131072, help="--stack: context in tokens")
+    ap.add_argument("--batch", type=int, default=4, help="--stack: sequences")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.stack is not None and args.impl == "ours":
+        run_stack(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

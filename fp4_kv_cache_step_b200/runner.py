@@ -69,7 +69,8 @@ class DeviceWorkload:
             self.args.append(csa2.layer_args(
                 self.q[layer], self.nvalid, self.out[layer], w.K, w.softmax_scale,
                 idx_q=self.idx_q[layer], idx_w=self.idx_w[layer], lse=self.lse[layer], N=N,
-                emit_pool=(mode == wl.FULL and w.C > 0),
+                emit_pool=(0 if mode != wl.FULL or w.C == 0 else
+                           (2 if w.pool_block == 8 else 1)),
                 use_pool=(mode == wl.REINDEX and w.C > 0)))
         need = max(csa2.layer_step_workspace_bytes(m, a, self.shared)
                    for m, a in zip(w.modes, self.args))
@@ -85,3 +86,18 @@ class DeviceWorkload:
             if snapshot_topk:
                 self.topk_per_layer[layer] = self.topk.clone()
         return self.out, self.lse
+
+
+class DeviceStack:
+    """The model's CSA2 layers (workloads.production_stack) on one GPU: one
+    DeviceWorkload per cache-sharing segment (three encoder groups, the
+    decoder), run in model order by `step()`."""
+
+    def __init__(self, stack: wl.Stack, device="cuda"):
+        self.stack = stack
+        self.segments = [DeviceWorkload(w, device) for w in stack.segments]
+
+    def step(self, snapshot_topk: bool = False):
+        for seg, layer in self.stack.layers:
+            self.segments[seg].step([layer], snapshot_topk=snapshot_topk)
+        return [(d.out, d.lse) for d in self.segments]

@@ -20,6 +20,16 @@ benchmark and the parity tests use):
    4:1 compression, each query sees entries whose 4 tokens are all at or
    before its own position
 
+The model's own shapes ("Model Setup Numbers Without Jargon" in "Detailed
+Notes On DeepSeek V4 Point 1 Flash In Simple Words"; mengman.github.io 3.3,
+3.4) as a layer stack, `production_stack(T, B)`: of the 40 layers the first 2
+use only the sliding window (no CSA2 step); 18 encoder layers at 2 tokens per
+entry form three groups [FULL + 5 REUSE], each FULL building its own main KV
+and indexer keys; 20 decoder layers at 1 token per entry form [FULL + 3 REUSE]
+and four [REINDEX + 3 REUSE] over the decoder FULL's cache, that FULL emitting
+the blockwise pool (2048 blocks of 8) which the REINDEX layers score; top-512,
+indexer 32 heads x 128, 64 query heads of 512.
+
 Values: main KV ~ N(0, 1) (quantised by the library), queries ~ N(0, 1)/sqrt(512)
 rounded to bf16, indexer queries and keys integers uniform in [-4, 4] stored
 as E4M3, head weights integers uniform in [1, 4].
@@ -51,6 +61,7 @@ class Workload:
     K: int
     D: int = 512
     C: int = 0                      # candidate pool size emitted by FULL (0 = none)
+    pool_block: int = 1             # 1: the top-C entries; 8: the blockwise pool, C/8 blocks
     modes: Tuple[str, ...] = (FULL,)
     lengths: str = "all"            # "all" | "uniform" | "chunk_end"
     len_lo: int = 0
@@ -169,6 +180,46 @@ def idx_q(w: Workload, layer: int = 0, rows=None) -> np.ndarray:
 
 def idx_w(w: Workload, layer: int = 0, rows=None) -> np.ndarray:
     return _stack(lambda b: idx_w_row(w, layer, b), list(range(w.B)) if rows is None else list(rows))
+
+
+# ------------------------------------------------------------ the model's stack
+PROD_HQ, PROD_HI, PROD_DI, PROD_K = 64, 32, 128, 512
+PROD_POOL_BLOCKS, PROD_POOL_BLOCK = 2048, 8
+PROD_SWA_ONLY_LAYERS = 2
+PROD_ENCODER_GROUPS = 3                             # [FULL + 5 REUSE] each, 2 tokens per entry
+PROD_DECODER_GROUPS = 5                             # [FULL|REINDEX + 3 REUSE], 1 token per entry
+
+
+@dataclasses.dataclass(frozen=True)
+class Stack:
+    """The CSA2 layers of the model's 40 in order, as segments that each share
+    one main KV and indexer-key cache: `segments[i]` is a Workload whose
+    `modes` are its layers; `layers` lists (segment, layer in segment) in
+    model order; `swa_only` counts the leading layers with no CSA2 step."""
+    segments: Tuple[Workload, ...]
+    layers: Tuple[Tuple[int, int], ...]
+    swa_only: int
+
+
+def production_stack(T: int, B: int, seed: int = 50, Hq: int = PROD_HQ, Hi: int = PROD_HI,
+                     Di: int = PROD_DI, K: int = PROD_K,
+                     pool_blocks: int = PROD_POOL_BLOCKS) -> Stack:
+    """The model's layer schedule for one decode step at context T tokens
+    (T even, T/2 a multiple of 64): encoder caches of T/2 entries (2 tokens
+    per entry, all visible to the newest query), a decoder cache of T entries."""
+    if T % 128 != 0:
+        raise ValueError("T must be a multiple of 128")
+    segs = []
+    for g in range(PROD_ENCODER_GROUPS):
+        segs.append(Workload("prod_encoder_group%d" % g, seed + g, B=B, Tq=1, N=T // 2, Hq=Hq,
+                             Hi=Hi, Di=Di, K=K, modes=(FULL,) + (REUSE,) * 5))
+    dec_modes = (FULL, REUSE, REUSE, REUSE) + (REINDEX, REUSE, REUSE, REUSE) * (
+        PROD_DECODER_GROUPS - 1)
+    segs.append(Workload("prod_decoder", seed + PROD_ENCODER_GROUPS, B=B, Tq=1, N=T, Hq=Hq, Hi=Hi,
+                         Di=Di, K=K, C=pool_blocks * PROD_POOL_BLOCK,
+                         pool_block=PROD_POOL_BLOCK, modes=dec_modes))
+    layers = tuple((i, l) for i, w in enumerate(segs) for l in range(len(w.modes)))
+    return Stack(tuple(segs), layers, PROD_SWA_ONLY_LAYERS)
 
 
 def small(name="small", seed=100, B=2, Tq=1, N=1024, Hq=8, Hi=4, Di=64, K=64, D=512, C=0,
