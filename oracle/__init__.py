@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.or_fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P]
         L.or_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, D, P, P]
         L.or_block_pool.argtypes = [P, I, I, P, I, I, P]
+        L.or_swa_sparse_attn.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, D, P, P]
         L.or_index_score.argtypes = [P, P, P, I, I, I, I, I, P, P, I, P]
         L.or_topk.argtypes = [P, I, I, P, P, I, P]
         L.or_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, I, I, D, P, P]
@@ -75,7 +76,7 @@ def lib() -> ctypes.CDLL:
         for f in (L.or_fp4_kv_pack, L.or_fp4_kv_unpack, L.or_index_score, L.or_topk,
                   L.or_sparse_attn, L.or_dense_attn, L.or_layer_step, L.or_fp4_kv_pack_g16,
                   L.or_fp4_kv_unpack_g16, L.or_fp4_kv_append_g16, L.or_sparse_attn_g16,
-                  L.or_block_pool):
+                  L.or_block_pool, L.or_swa_sparse_attn):
             f.restype = I
         _lib = L
     return _lib
@@ -262,6 +263,32 @@ def sparse_attn(q_bf16, packed, scale, idx, softmax_scale):
     _check(lib().or_sparse_attn(_ptr(q_bf16), _ptr(packed), _ptr(scale), _ptr(idx), B, Tq, Hq,
                                 D, N, K, float(softmax_scale), _ptr(out), _ptr(lse)),
            "or_sparse_attn")
+    return out, lse
+
+
+SWA_WINDOW = 128
+
+
+def swa_sparse_attn(q_bf16, packed, scale, idx, swa_kv, swa_n, softmax_scale, W=SWA_WINDOW):
+    """Sparse attention plus the sliding-window branch, one softmax over both:
+    swa_kv u8 (E4M3) [B][Tw][D], swa_n i32 [B][Tq] (query sees window tokens
+    [max(0, swa_n - W), swa_n))."""
+    q_bf16 = _c(q_bf16, np.uint16)
+    packed = _c(packed, np.uint8)
+    scale = _c(scale, np.uint8)
+    idx = _c(idx, np.int32)
+    swa_kv = _c(swa_kv, np.uint8)
+    swa_n = _c(swa_n, np.int32)
+    B, Tq, Hq, D = q_bf16.shape
+    N = packed.shape[1]
+    K = idx.shape[-1]
+    Tw = swa_kv.shape[1]
+    out = np.zeros((B, Tq, Hq, D), np.float64)
+    lse = np.zeros((B, Tq, Hq), np.float64)
+    _check(lib().or_swa_sparse_attn(_ptr(q_bf16), _ptr(packed), _ptr(scale), _ptr(idx),
+                                    _ptr(swa_kv), _ptr(swa_n), B, Tq, Hq, D, N, K, Tw, int(W),
+                                    float(softmax_scale), _ptr(out), _ptr(lse)),
+           "or_swa_sparse_attn")
     return out, lse
 
 

@@ -429,6 +429,57 @@ static double kv_source_value(const kv_source* src, int b, int n, int c) {
     return g16_value(src->kv_packed, src->N, src->D, b, n, c);
 }
 
+/* Softmax attention of every head of query row `row` over the n value rows
+ * v[0..n) (each serving as key and value): out = sum_k softmax(l)_k v_k with
+ * l_k = softmax_scale * q . v_k; lse = log sum_k exp(l_k). No row: out = 0,
+ * lse = -inf. `logit` has room for n values. */
+static void attend_rows(const uint16_t* q, size_t row, int Hq, int D, const double* v, int n,
+                        double softmax_scale, double* logit, double* out, double* lse) {
+    for (int h = 0; h < Hq; ++h) {
+        const uint16_t* qh = q + (row * Hq + h) * D;
+        double* oh = out + (row * Hq + h) * D;
+        if (n == 0) {
+            for (int c = 0; c < D; ++c) oh[c] = 0.0;
+            if (lse) lse[row * Hq + h] = -INFINITY;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int k = 0; k < n; ++k) {
+            double dot = 0.0;
+            for (int c = 0; c < D; ++c) dot += or_bf16_value(qh[c]) * v[(size_t)k * D + c];
+            logit[k] = softmax_scale * dot;
+            if (logit[k] > m) m = logit[k];
+        }
+        double z = 0.0;
+        for (int k = 0; k < n; ++k) {
+            logit[k] = exp(logit[k] - m); /* now the unnormalised weight */
+            z += logit[k];
+        }
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < n; ++k) acc += logit[k] * v[(size_t)k * D + c];
+            oh[c] = acc / z;
+        }
+        if (lse) lse[row * Hq + h] = m + log(z);
+    }
+}
+
+/* The selected main-KV rows of query row (b, row), dequantised into v; returns
+ * their number, or -1 for an index outside [-1, N). */
+static int gather_selected(const kv_source* src, const int32_t* topk, int b, size_t row, int D,
+                           int N, int K, double* v) {
+    int n = 0;
+    for (int k = 0; k < K; ++k) {
+        int32_t id = topk[row * K + k];
+        if (id < 0) continue;
+        if (id >= N) return -1;
+        for (int c = 0; c < D; ++c)
+            v[(size_t)n * D + c] = kv_source_value(src, b, id, c);
+        ++n;
+    }
+    return n;
+}
+
 static int sparse_attn_rows(const uint16_t* q, const kv_source* src, const int32_t* topk,
                             int B, int Tq, int Hq, int D, int N, int K,
                             double softmax_scale, double* out, double* lse) {
@@ -439,44 +490,52 @@ static int sparse_attn_rows(const uint16_t* q, const kv_source* src, const int32
     for (int b = 0; b < B && rc == OR_OK; ++b) {
         for (int t = 0; t < Tq && rc == OR_OK; ++t) {
             size_t row = (size_t)b * Tq + t;
-            /* dequantise the selected rows */
-            int n = 0;
-            for (int k = 0; k < K; ++k) {
-                int32_t id = topk[row * K + k];
-                if (id < 0) continue;
-                if (id >= N) { rc = OR_BAD_INDEX; break; }
+            int n = gather_selected(src, topk, b, row, D, N, K, v);
+            if (n < 0) { rc = OR_BAD_INDEX; break; }
+            attend_rows(q, row, Hq, D, v, n, softmax_scale, logit, out, lse);
+        }
+    }
+    free(v);
+    free(logit);
+    return rc;
+}
+
+/* The sliding-window branch beside the sparse set ("Detailed Notes On
+ * DeepSeek V4 Point 1 Flash In Simple Words": every layer also looks at the
+ * recent tokens through sliding-window attention, window 128, its memory kept
+ * at 8 bits; mengman.github.io 3.3, 3.5). How the two branches combine is not
+ * stated; here one softmax runs over the union of the selected main rows and
+ * the window's tokens. The window memory of row b is swa_kv[b][0..Tw) (one
+ * E4M3 row of D values per token, no scale, serving as key and value); query
+ * (b, t) sees its tokens [max(0, swa_n - W), swa_n), swa_n = swa_n[b][t]. */
+int or_swa_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                       const int32_t* topk, const uint8_t* swa_kv, const int32_t* swa_n,
+                       int B, int Tq, int Hq, int D, int N, int K, int Tw, int W,
+                       double softmax_scale, double* out, double* lse) {
+    if (!q || !kv_packed || !kv_scale || !topk || !swa_kv || !swa_n || !out || B < 0 ||
+        Tq < 0 || Hq <= 0 || D <= 0 || N < 0 || K <= 0 || Tw < 0 || W < 0)
+        return OR_BAD_ARG;
+    if (N % OR_BLOCK != 0 || D % 2 != 0) return OR_BAD_ARG;
+    e4m3_table_init();
+    kv_source src = {kv_packed, kv_scale, N, D};
+    double* v = (double*)malloc(sizeof(double) * ((size_t)K + (size_t)W) * D);
+    double* logit = (double*)malloc(sizeof(double) * ((size_t)K + (size_t)W > 0 ? (size_t)K + W : 1));
+    if (!v || !logit) { free(v); free(logit); return OR_BAD_ARG; }
+    int rc = OR_OK;
+    for (int b = 0; b < B && rc == OR_OK; ++b) {
+        for (int t = 0; t < Tq && rc == OR_OK; ++t) {
+            size_t row = (size_t)b * Tq + t;
+            int n = gather_selected(&src, topk, b, row, D, N, K, v);
+            if (n < 0) { rc = OR_BAD_INDEX; break; }
+            int hi = swa_n[row];
+            if (hi < 0 || hi > Tw) { rc = OR_BAD_ARG; break; }
+            int lo = hi - W > 0 ? hi - W : 0;
+            for (int j = lo; j < hi; ++j) {
                 for (int c = 0; c < D; ++c)
-                    v[(size_t)n * D + c] = kv_source_value(src, b, id, c);
+                    v[(size_t)n * D + c] = g_e4m3_table[swa_kv[((size_t)b * Tw + j) * D + c]];
                 ++n;
             }
-            if (rc != OR_OK) break;
-            for (int h = 0; h < Hq; ++h) {
-                const uint16_t* qh = q + (row * Hq + h) * D;
-                double* oh = out + (row * Hq + h) * D;
-                if (n == 0) {
-                    for (int c = 0; c < D; ++c) oh[c] = 0.0;
-                    if (lse) lse[row * Hq + h] = -INFINITY;
-                    continue;
-                }
-                double m = -INFINITY;
-                for (int k = 0; k < n; ++k) {
-                    double dot = 0.0;
-                    for (int c = 0; c < D; ++c) dot += or_bf16_value(qh[c]) * v[(size_t)k * D + c];
-                    logit[k] = softmax_scale * dot;
-                    if (logit[k] > m) m = logit[k];
-                }
-                double z = 0.0;
-                for (int k = 0; k < n; ++k) {
-                    logit[k] = exp(logit[k] - m); /* now the unnormalised weight */
-                    z += logit[k];
-                }
-                for (int c = 0; c < D; ++c) {
-                    double acc = 0.0;
-                    for (int k = 0; k < n; ++k) acc += logit[k] * v[(size_t)k * D + c];
-                    oh[c] = acc / z;
-                }
-                if (lse) lse[row * Hq + h] = m + log(z);
-            }
+            attend_rows(q, row, Hq, D, v, n, softmax_scale, logit, out, lse);
         }
     }
     free(v);

@@ -109,6 +109,14 @@ int or_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows, const int32_t*
                        int B, int Tq, int Hq, int D, int N, int K,
                        double softmax_scale, double* out, double* lse);
 
+/* Sparse attention with the sliding-window branch: one softmax over the
+ * selected main rows and the window tokens [max(0, swa_n[b][t] - W),
+ * swa_n[b][t]) of swa_kv[b] (u8 E4M3 [B][Tw][D], no scale, key = value). */
+int or_swa_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
+                       const int32_t* topk, const uint8_t* swa_kv, const int32_t* swa_n,
+                       int B, int Tq, int Hq, int D, int N, int K, int Tw, int W,
+                       double softmax_scale, double* out, double* lse);
+
 /* Softmax attention of every head over all entries j < nvalid[b][t] (dense). */
 int or_dense_attn(const uint16_t* q, const uint8_t* kv_packed, const uint8_t* kv_scale,
                   const int32_t* nvalid, int B, int Tq, int Hq, int D, int N,
