@@ -32,6 +32,7 @@ if ROOT not in sys.path:
 
 METRIC = "CSA2 decode layer-steps/s at 128K ctx; achieved HBM GB/s vs 8 TB/s peak"
 UNIT = "layer-steps/s"
+DEFAULT_WORKLOAD = "decode_128k_full"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -197,7 +198,7 @@ def run_ours(args):
         dist.barrier()
     csa2.load()
 
-    w = rank_workload(wl.CONFIGS[args.config], rank)
+    w = rank_workload(wl.WORKLOADS[args.workload], rank)
     dw = DeviceWorkload(w, dev)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -474,7 +475,7 @@ def run_reference(args):
     from fp4_kv_cache_step_b200 import workloads as wl
     import oracle
     oracle.build()
-    w = wl.CONFIGS[args.config]
+    w = wl.WORKLOADS[args.workload]
     for i in range(args.warmup):
         oracle_layer_steps(w, [i % w.B])
     secs = [oracle_layer_steps(w, [i % w.B]) for i in range(args.steps)]
@@ -561,7 +562,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="workload name (fp4_kv_cache_step_b200.workloads.WORKLOADS)")
     ap.add_argument("--cpu-sample-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-bound", default="tensor", choices=["tensor", "hbm"])

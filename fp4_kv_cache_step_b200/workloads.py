@@ -7,18 +7,19 @@ own dtype casts (float32 -> bfloat16, small integers -> float8_e4m3fn). Every
 tensor has its own stream keyed by (seed, tensor tag, layer, batch row), so a
 test can regenerate one batch row of a large workload without the rest.
 
-Workloads (sizes and value distributions of the five configurations the
-benchmark and the parity tests use):
+Workloads (sizes and value distributions the benchmark and the parity tests
+use), by name in WORKLOADS:
 
-0  tiny decode, FULL: B=1, N=4096, 16 query heads, indexer 4 x 64, top-256
-1  decode at 128K tokens, FULL: B=32, N=32768, 64 heads, indexer 64 x 128,
-   top-2048, lengths uniform in [16384, 32768]
-2  4-layer stack FULL, REINDEX, REUSE, REUSE: B=16, N=16384
-3  1M tokens, FULL emitting a top-8192 pool, then REINDEX inside the pool:
-   B=4, N=262144
-4  prefill chunk, FULL: 4096 query tokens at the end of N=65536 entries at
-   4:1 compression, each query sees entries whose 4 tokens are all at or
-   before its own position
+TINY_DECODE    tiny decode, FULL: B=1, N=4096, 16 query heads, indexer 4 x 64,
+               top-256
+DECODE_128K    decode at 128K tokens, FULL: B=32, N=32768, 64 heads, indexer
+               64 x 128, top-2048, lengths uniform in [16384, 32768]
+STACK_4        4-layer stack FULL, REINDEX, REUSE, REUSE: B=16, N=16384
+HIER_1M        1M tokens, FULL emitting a top-8192 pool, then REINDEX inside
+               the pool: B=4, N=262144
+PREFILL_CHUNK  prefill chunk, FULL: 4096 query tokens at the end of N=65536
+               entries at 4:1 compression, each query sees entries whose 4
+               tokens are all at or before its own position
 
 The model's own shapes ("Model Setup Numbers Without Jargon" in "Detailed
 Notes On DeepSeek V4 Point 1 Flash In Simple Words"; mengman.github.io 3.3,
@@ -76,17 +77,16 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-CONFIGS = {
-    0: Workload("tiny_decode_full", 0, B=1, Tq=1, N=4096, Hq=16, Hi=4, Di=64, K=256),
-    1: Workload("decode_128k_full", 1, B=32, Tq=1, N=32768, Hq=64, Hi=64, Di=128, K=2048,
-                lengths="uniform", len_lo=16384, len_hi=32768),
-    2: Workload("stack_full_reindex_reuse_reuse", 2, B=16, Tq=1, N=16384, Hq=64, Hi=64, Di=128,
-                K=2048, modes=(FULL, REINDEX, REUSE, REUSE)),
-    3: Workload("hier_1m_full_pool_reindex", 3, B=4, Tq=1, N=262144, Hq=64, Hi=64, Di=128,
-                K=2048, C=8192, modes=(FULL, REINDEX)),
-    4: Workload("prefill_chunk_4096_full", 4, B=1, Tq=4096, N=65536, Hq=64, Hi=64, Di=128,
-                K=2048, lengths="chunk_end"),
-}
+TINY_DECODE = Workload("tiny_decode_full", 0, B=1, Tq=1, N=4096, Hq=16, Hi=4, Di=64, K=256)
+DECODE_128K = Workload("decode_128k_full", 1, B=32, Tq=1, N=32768, Hq=64, Hi=64, Di=128, K=2048,
+                       lengths="uniform", len_lo=16384, len_hi=32768)
+STACK_4 = Workload("stack_full_reindex_reuse_reuse", 2, B=16, Tq=1, N=16384, Hq=64, Hi=64,
+                   Di=128, K=2048, modes=(FULL, REINDEX, REUSE, REUSE))
+HIER_1M = Workload("hier_1m_full_pool_reindex", 3, B=4, Tq=1, N=262144, Hq=64, Hi=64, Di=128,
+                   K=2048, C=8192, modes=(FULL, REINDEX))
+PREFILL_CHUNK = Workload("prefill_chunk_4096_full", 4, B=1, Tq=4096, N=65536, Hq=64, Hi=64,
+                         Di=128, K=2048, lengths="chunk_end")
+WORKLOADS = {w.name: w for w in (TINY_DECODE, DECODE_128K, STACK_4, HIER_1M, PREFILL_CHUNK)}
 
 
 def _rng(seed: int, *key: int) -> np.random.Generator:

@@ -33,9 +33,11 @@ def _run(w):
     return dw
 
 
-@pytest.mark.parametrize("cfg,rows", [(1, [0, 13, 31]), (2, [0, 15]), (3, [2])])
-def test_full_size_config(cfg, rows):
-    w = wl.CONFIGS[cfg]
+@pytest.mark.parametrize("name,rows", [("decode_128k_full", [0, 13, 31]),
+                                       ("stack_full_reindex_reuse_reuse", [0, 15]),
+                                       ("hier_1m_full_pool_reindex", [2])])
+def test_full_size_workload(name, rows):
+    w = wl.WORKLOADS[name]
     dw = _run(w)
     _check_stack(w, dw, _oracle_stack(w, rows), rows)
     # every row's indices are valid: ascending, inside [0, nvalid), -1 only as padding
@@ -51,7 +53,7 @@ def test_full_size_config(cfg, rows):
 
 
 def test_full_size_prefill_chunk_sampled_queries():
-    w = wl.CONFIGS[4]
+    w = wl.PREFILL_CHUNK
     dw = _run(w)
     tsel = [0, 1, 3, 4, 2047, 4095]
     packed, sc = oracle.fp4_kv_pack(wl.kv(w, rows=[0]))

@@ -277,7 +277,7 @@ def _check_stack(w, dw, want, rows):
 
 
 def test_layer_step_config0_full():
-    w = wl.CONFIGS[0]
+    w = wl.TINY_DECODE
     dw = DeviceWorkload(w)
     dw.step(snapshot_topk=True)
     csa2.check_device_errors()

@@ -30,7 +30,7 @@ def _init(rank, world, port, timeout_s=20):
 def _worker_reduce(rank, world, port, q):
     _init(rank, world, port)
     try:
-        w = bench.rank_workload(wl.CONFIGS[1], rank)
+        w = bench.rank_workload(wl.DECODE_128K, rank)
         got = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
         seeds = [None] * world
         dist.all_gather_object(seeds, w.seed)

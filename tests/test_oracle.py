@@ -432,15 +432,15 @@ def test_layer_step_full_matches_composed_calls(oracle_lib):
 
 # ----------------------------------------------------------------- workloads
 def test_workloads_are_seeded_and_shaped(facts):
-    w = wl.CONFIGS[4]
+    w = wl.PREFILL_CHUNK
     nv = wl.nvalid(w)
     assert nv.shape == (1, 4096) and nv.min() == 65536 - 1024 and nv.max() == 65536
     assert nv[0, 0] == 64512 and nv[0, 3] == 64513 and nv[0, 4095] == 65536
-    w1 = wl.CONFIGS[1]
+    w1 = wl.DECODE_128K
     n1 = wl.nvalid(w1)
     assert n1.shape == (32, 1) and n1.min() >= 16384 and n1.max() <= 32768
     assert np.array_equal(n1, wl.nvalid(w1))
-    w0 = wl.CONFIGS[0]
+    w0 = wl.TINY_DECODE
     a, b = wl.idx_q(w0), wl.idx_q(w0)
     assert np.array_equal(a, b) and a.shape == (1, 1, 4, 64)
     vals = torch.from_numpy(a).view(torch.float8_e4m3fn).float().numpy()
