@@ -31,8 +31,8 @@
  *    16-bit patterns (uint16_t), E4M3 values as bytes.
  *  - Packed FP4: byte c/2 of an entry holds channel c, low nibble = even c.
  *    Scales: one E4M3 byte per channel per 64-entry block,
- *    kv_scale[b][n/64][c] (the block-scale layout the benchmark
- *    configurations state). The pages' own layout, one E4M3 scale per 16
+ *    kv_scale[b][n/64][c] (the block-scale layout of the benchmark
+ *    workloads). The pages' own layout, one E4M3 scale per 16
  *    channels of an entry, has its own calls (*_g16): an entry is one row of
  *    D/2 code bytes followed by D/16 scale bytes, kv_rows[b][n][D/2 + D/16].
  *  - Pointers must be 16-byte aligned; D must be 512 for attention; N must be a
