@@ -165,3 +165,24 @@ def test_layer_step_blockwise_pool_needs_a_multiple_of_eight(lib):
     args.emit_pool = 3
     rc = lib.csa2_layer_step(ctypes.byref(args), 0, ctypes.byref(sh), None, 0, None)
     assert _status(rc) == "INVALID_ARG"
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    """A C caller needs nothing but the header: it compiles as strict C99 with
+    no CUDA headers, and every declared call can be referenced."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = tmp_path / "use_header.c"
+    src.write_text(
+        '#include "csa2.h"\n'
+        "typedef void (*any_fn)(void);\n"
+        "any_fn table[] = {\n" + "".join("  (any_fn)%s,\n" % n for n in names) + "};\n"
+        "int main(void) { return table[0] == 0; }\n")
+    rc = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-c", str(src), "-I", os.path.dirname(HEADER),
+                         "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert rc.returncode == 0, rc.stderr
