@@ -124,7 +124,8 @@ CSA2_API csa2_status fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8
 
 /* fp4_kv_unpack_g16 -- exact dequantisation of the 16-channel layout:
  * out[b][n][c] = e2m1(code) * e4m3(scale of group c / 16).
- *   out      float [B][N][D]              output */
+ *   out      float [B][N][D]              output (every value exact in fp32)
+ * Requires D % 128 == 0, as fp4_kv_pack_g16. */
 CSA2_API csa2_status fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, float* out,
                                        csa2_stream_t stream);
 
@@ -139,6 +140,8 @@ CSA2_API csa2_status fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int
  *                                         CSA2_ERR_DEVICE_INDEX recorded; the
  *                                         positions of one b must differ
  *   kv_rows  uint8 [B][N][D/2 + D/16]     updated in place
+ * Requires D % 128 == 0, T >= 0. A NaN or infinity records CSA2_ERR_NONFINITE
+ * (the row is still written).
  * ------------------------------------------------------------------------ */
 CSA2_API csa2_status fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, int T,
                                        int N, int D, uint8_t* kv_rows, csa2_stream_t stream);
