@@ -93,17 +93,8 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// Same, with each descriptor given as its low word (start address and leading
-// offset: advancing it by (bytes >> 4) cannot carry out, shared-memory
+// One MMA with each descriptor given as its low word (start address and
+// leading offset: advancing it by (bytes >> 4) cannot carry out, shared-memory
 // addresses being below 2^18) and a common high word.
 __device__ __forceinline__ void mma_f16_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi_a,
                                            uint32_t hi_b, uint32_t idesc, uint32_t acc) {
