@@ -1,25 +1,36 @@
 #!/usr/bin/env python
-"""Benchmark: CSA2 decode layer step at 128K tokens of context (FULL mode).
+"""Benchmark of the CSA2 layer step over an FP4 main KV cache.
 
-Workload "decode_128k_full": batch 32, one query token each, N = 32768 FP4
-main-KV entries of dim 512 (128K tokens at 4:1 compression), 64 bf16 query
+Default workload "decode_128k_full": batch 32, one query token each, N = 32768
+FP4 main-KV entries of dim 512 (128K tokens at 4:1 compression), 64 bf16 query
 heads, indexer 64 heads x 128 with integer E4M3 values, top-2048, lengths
 uniform in [16384, 32768]. One step = one pass of the whole hot path over the
-batch: indexer scores -> top-K -> gather + FP4 dequant + sparse attention (+
-split combine). The FP4 cache is built once before timing (a cache is built
-when tokens arrive, not per step). Inputs are resident in HBM; L2 is flushed
-between timed steps (a 256 MiB write, then a 256 MiB read so that the flush's
-dirty lines are written back there), outside the timed events.
+batch: indexer scores -> top-K -> gather + FP4 dequant + sparse attention. The
+FP4 cache is built once before timing (a cache is built when tokens arrive, not
+per step). Inputs are resident in HBM; L2 is flushed between timed steps (a
+256 MiB write, then a 256 MiB read so the flush's dirty lines are written back
+there), outside the timed events.
 
-Prints one JSON line. With --impl reference it times the CPU oracle on a
-bounded sample of the same workload instead.
+The other workloads (--workload NAME, see fp4_kv_cache_step_b200.workloads)
+print their own line: the tiny decode, the 4-layer FULL/REINDEX/REUSE/REUSE
+stack (per layer and per stack), the 1M-token hierarchical pair (FULL emitting
+a top-8192 pool, REINDEX inside it) and the 4096-query prefill chunk (whose
+indexer is reported against the FP8 tensor peak). --stack production times the
+model's own 38 CSA2 layers.
+
+Prints one JSON line. With --impl reference it times the CPU oracle on the same
+workload instead (the oracle is the only other implementation: the pages print
+no code).
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
+import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import sys
 import time
@@ -36,6 +47,35 @@ DEFAULT_WORKLOAD = "decode_128k_full"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0           # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+DTYPE = "e4m3 x e4m3 and f16 x f16 tensor-core products, f32 accumulation (FP4/E4M3 storage, bf16 out)"
+CSRC = os.path.join(ROOT, "fp4_kv_cache_step_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+
+# the sources each timed kernel is built from (its captured counters hold while they are unchanged)
+KERNEL_SOURCES = {
+    "score": ("score_tc.cu", "sm100.cuh", "common.cuh"),
+    "topk": ("topk.cu", "common.cuh"),
+    "attn": ("attn_tc.cu", "attn.cu", "sm100.cuh", "common.cuh"),
+}
+
+
+def workload_metric(w):
+    """(metric, unit) of a workload's line: one 'step' is one pass of its whole
+    mode schedule over its batch."""
+    if w.name in ("decode_128k_full",):
+        return METRIC, UNIT
+    if w.name == "tiny_decode_full":
+        return "CSA2 decode layer-steps/s, tiny decode (B=1, N=4096)", UNIT
+    if w.name == "stack_full_reindex_reuse_reuse":
+        return "CSA2 4-layer stack steps/s (FULL, REINDEX, REUSE, REUSE; B=16, N=16384)", \
+            "stack-steps/s"
+    if w.name == "hier_1m_full_pool_reindex":
+        return "CSA2 hierarchical steps/s at 1M tokens (FULL + top-8192 pool, REINDEX in pool)", \
+            "hier-steps/s"
+    if w.name == "prefill_chunk_4096_full":
+        return "CSA2 prefill-chunk layer-steps/s (4096 queries over 65536 entries)", UNIT
+    return "CSA2 %s steps/s" % w.name, "steps/s"
 
 
 def dist_env():
@@ -59,25 +99,37 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def profiled_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
-    when the kernel's source has changed since the counters were taken."""
-    import hashlib
-    import re
-    if kernel != "attn":
-        return None
-    src = os.path.join(ROOT, "fp4_kv_cache_step_b200", "csrc", "attn_tc.cu")
-    prof = os.path.join(ROOT, "profiles", "decode_128k_step_kernels.md")
+def sources_sha1(kernel: str) -> str:
+    h = hashlib.sha1()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel: str, workload: str, units: float):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    record (profiles/kernel_traffic.json), or (None, why) when there is no
+    capture of the kernel's current sources. A capture on a smaller case of the
+    same kernel is scaled by the units processed (valid keys for the scorer,
+    selected entries for the attention)."""
     try:
-        text = open(prof).read()
-        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
-        m_sha = re.search(r"attn_tc\.cu sha1 at capture: ([0-9a-f]{40})", text)
-        m_b = re.search(r"= ([0-9,]+) bytes", text)
-        if m_sha and m_b and m_sha.group(1) == sha:
-            return int(m_b.group(1).replace(",", ""))
-    except OSError:
-        pass
-    return None
+        with open(TRAFFIC_FILE) as f:
+            recs = json.load(f)["captures"]
+    except (OSError, ValueError, KeyError):
+        return None, "no ncu record"
+    sha = sources_sha1(kernel)
+    best = None
+    for r in recs:
+        if r.get("kernel") != kernel or r.get("sources_sha1") != sha:
+            continue
+        if r.get("workload") == workload:
+            return float(r["dram_bytes_per_launch"]), "ncu capture of this workload"
+        best = best or r
+    if best is not None and best.get("units"):
+        return float(best["dram_bytes_per_launch"]) * units / float(best["units"]), \
+            "ncu capture of %s scaled by units (%s)" % (best["workload"], best.get("unit_kind"))
+    return None, "sources changed since the last ncu capture"
 
 
 def measured_peaks():
@@ -85,37 +137,94 @@ def measured_peaks():
     try:
         with open(path) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured (MEASURED_PEAKS.json)"}
     except Exception:
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def fp8_matmul_peak_live(dev, n: int = 8192, reps: int = 10) -> float:
+    """Dense E4M3 GEMM throughput of torch._scaled_mm (cuBLASLt) on this GPU,
+    best of `reps`, TFLOP/s: context for the FP8 roofline of the prefill indexer."""
+    import torch
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------- algorithmic bytes
-def algorithmic_bytes(w, nvalid: np.ndarray, topk: np.ndarray) -> dict:
-    """Bytes each kernel must move at least, from the realised lengths and the
-    selected indices (distinct 64-entry scale blocks per sequence)."""
+def layer_accounting(w, mode: str, nvalid: np.ndarray, topk: np.ndarray, cand=None,
+                     pooled: bool = False, emit_pool: bool = False) -> dict:
+    """Bytes (and flops) each kernel of one layer must move at least, from the
+    realised lengths and selections: the scorer reads every visible key (or the
+    pool's keys) and the indexer query, and writes one score per key; the top-K
+    reads the scores and writes K ids; the attention reads the selected packed
+    rows, each distinct 64-entry scale row once, the queries and the ids, and
+    writes the outputs. 'metric' is what the step must bring from HBM: keys,
+    indexer queries, selected rows, scale rows, queries and outputs (scores and
+    ids are intermediates)."""
     rows = w.B * w.Tq
-    nv = nvalid.reshape(-1).astype(np.int64)
     tk = topk.reshape(rows, w.K)
-    sel = (tk >= 0).sum(axis=1).astype(np.int64)
-    blocks = np.array([np.unique(r[r >= 0] // 64).size for r in tk], np.int64)
-    idx_k = int(nv.sum()) * w.Di
-    idx_qw = rows * (w.Hi * w.Di + 4 * w.Hi)
-    scores = int(nv.sum()) * 4
-    kv_rows = int(sel.sum()) * (w.D // 2)
-    scale_rows = int(blocks.sum()) * w.D
+    sel = int((tk >= 0).sum())
+    blocks = int(sum(np.unique(r[r >= 0] // 64).size for r in tk))
     q_out = 2 * rows * w.Hq * w.D * 2
     idx = rows * w.K * 4
-    return {
-        "score": idx_k + idx_qw + scores,
-        "topk": scores + idx,
-        "attn": kv_rows + scale_rows + q_out + idx,
-        # the 16-channel layout: codes and their own scales in one row per entry
-        "attn_g16": int(sel.sum()) * (w.D // 2 + w.D // 16) + q_out + idx,
-        "step": idx_k + idx_qw + kv_rows + scale_rows + q_out,
-        "flops_score": int(nv.sum()) * w.Hi * w.Di * 2,
-        "flops_attn": int(sel.sum()) * w.Hq * w.D * 4,
-    }
+    attn = sel * (w.D // 2) + blocks * w.D + q_out + idx
+    acc = {"attn": attn, "attn_flops": sel * w.Hq * w.D * 4, "selected": sel,
+           "scale_blocks": blocks, "score": 0, "score_flops": 0, "topk": 0, "keys": 0,
+           "metric": sel * (w.D // 2) + blocks * w.D + q_out}
+    if mode == "REUSE":
+        return acc
+    idx_qw = rows * (w.Hi * w.Di + 4 * w.Hi)
+    if pooled:
+        c = cand.reshape(rows, -1)
+        keys = int((c >= 0).sum())
+        acc["score"] = keys * (w.Di + 4) + c.size * 4 + idx_qw
+        acc["topk"] = keys * 4 + c.size * 4 + idx
+    else:
+        keys = int(np.minimum(nvalid.reshape(-1).astype(np.int64), w.N).sum())
+        acc["score"] = keys * (w.Di + 4) + idx_qw
+        acc["topk"] = keys * 4 + idx + (rows * w.C * 4 if emit_pool else 0)
+    acc["keys"] = keys
+    acc["score_flops"] = keys * w.Hi * w.Di * 2
+    acc["metric"] += keys * w.Di + idx_qw
+    return acc
+
+
+def roofline(kernel: str, acc: dict, us: float, peaks: dict, fp8_peak: float) -> dict:
+    """The kernel against whichever roofline bounds it: HBM bytes at the measured
+    copy rate, or tensor-core flops at the measured peak of its dtype (the
+    scorer is E4M3: the bf16 peak times the nominal FP8/bf16 ratio; attention is
+    f16, at the bf16 peak)."""
+    byts = acc[kernel]
+    flops = acc.get(kernel + "_flops", 0)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    tpeak = fp8_peak if kernel == "score" else peaks["bf16_tflops"]
+    t_tc = flops / (tpeak * 1e12) if flops else 0.0
+    if t_tc > t_hbm:
+        ach = flops / (us * 1e-6) / 1e12
+        r = {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
+             "frac": ach / tpeak}
+    else:
+        ach = byts / (us * 1e-6) / 1e9
+        r = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": ach / peaks["hbm_gbs"]}
+    r.update({"kernel": kernel, "us": us, "algorithmic_bytes": byts, "flops": flops,
+              "hbm_frac": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]})
+    return r
 
 
 # --------------------------------------------------------------- clocks
@@ -178,6 +287,26 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our arm
+class L2Flush:
+    """Writes 256 MiB (evicting every line of the step's data), then reads
+    another 256 MiB so that the dirty flush lines are written back here,
+    outside the timed events, not by the next step's first kernel."""
+
+    def __init__(self, torch, dev):
+        self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self, i: int):
+        self.w.fill_(i & 0xff)
+        self.r.max()
+
+
+def _mode_flags(w, mode):
+    pooled = mode == "REINDEX" and w.C > 0
+    emit = mode == "FULL" and w.C > 0
+    return pooled, emit
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -199,18 +328,11 @@ def run_ours(args):
     csa2.load()
 
     w = rank_workload(wl.WORKLOADS[args.workload], rank)
+    metric, unit = workload_metric(w)
     dw = DeviceWorkload(w, dev)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
-
-    def flush_l2(i):
-        # write 256 MiB (evicts every line of the step's data), then read another
-        # 256 MiB so that the dirty flush lines are written back here, outside
-        # the timed events, not by the next step's first kernel
-        flush.fill_(i & 0xff)
-        flush_rd.max()
+    flush_l2 = L2Flush(torch, dev)
 
     def barrier():
         if world > 1:
@@ -239,89 +361,91 @@ def run_ours(args):
     ms_per_step = max_total_ms / args.steps
     value = world * args.steps / (max_total_ms / 1e3)
 
-    # ---- per-kernel timing: the same kernels through the individual calls
-    nsplit_ws = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K)
-    kern = {"score": [], "topk": [], "attn": [], "block_pool": []}
-    # the hierarchical indexer's blockwise pool (2048 blocks of 8), as a FULL
-    # decoder layer emits it right after its top-K, from the same scores
-    pool_out = torch.empty((w.B, w.Tq, 2048 * 8), dtype=torch.int32, device=dev)
-    pool_ws = torch.empty(max(int(csa2.load().csa2_block_pool_workspace_bytes(
-        w.B, w.Tq, w.N, 8, 2048)), 256), dtype=torch.uint8, device=dev)
-    scores = torch.empty((w.B, w.Tq, w.N), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(int(nsplit_ws), 256), dtype=torch.uint8, device=dev)
-    out = torch.empty_like(dw.out[0])
-    lse = torch.empty_like(dw.lse[0])
+    # ---- per layer (events between the layers of a step; L2 flushed between steps only,
+    # so a REINDEX layer may find the FULL layer's keys in L2, as it would in the model)
+    nl = len(w.modes)
+    layer_ms = [[] for _ in range(nl)]
     for i in range(args.warmup + args.steps):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         flush_l2(i)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)]
         evs[0].record(stream)
-        csa2.csa2_index_score(dw.idx_q[0], dw.idx_w[0], dw.idx_k, nvalid=dw.nvalid, out=scores)
-        evs[1].record(stream)
-        csa2.csa2_topk(scores, w.K, nvalid=dw.nvalid, out=dw.topk)
-        evs[2].record(stream)
-        e_pool = torch.cuda.Event(enable_timing=True)
-        csa2.csa2_block_pool(scores, dw.nvalid, 2048, 8, out=pool_out, workspace=pool_ws)
-        e_pool.record(stream)
-        flush_l2(i)
-        evs[3].record(stream)
-        csa2.csa2_sparse_attn(dw.q[0], dw.kv_packed, dw.kv_scale, dw.topk, w.softmax_scale,
-                              out=out, lse=lse, workspace=ws)
-        e4 = torch.cuda.Event(enable_timing=True)
-        e4.record(stream)
+        for l in range(nl):
+            dw.step([l])
+            evs[l + 1].record(stream)
         torch.cuda.synchronize()
         if i >= args.warmup:
-            kern["score"].append(evs[0].elapsed_time(evs[1]))
-            kern["topk"].append(evs[1].elapsed_time(evs[2]))
-            kern["attn"].append(evs[3].elapsed_time(e4))
-            kern["block_pool"].append(evs[2].elapsed_time(e_pool))
-    kern_us = {k: 1e3 * statistics.mean(v) for k, v in kern.items()}
-
+            for l in range(nl):
+                layer_ms[l].append(evs[l].elapsed_time(evs[l + 1]))
+    # the selections each layer used (for the byte counts)
+    dw.step(snapshot_topk=True)
+    torch.cuda.synchronize()
+    csa2.check_device_errors()
     nvalid = wl.nvalid(w)
-    ab = algorithmic_bytes(w, nvalid, dw.topk.cpu().numpy())
-    hbm_peak, tf_peak, peak_kind = measured_peaks()
-    dom = max(("score", "attn", "topk"), key=lambda k: kern_us[k])
-    if dom == "attn" and args.attn_bound == "tensor":
-        achieved = ab["flops_attn"] / (kern_us["attn"] * 1e-6) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
-                "frac": achieved / tf_peak}
-    else:
-        achieved = ab[dom] / (kern_us[dom] * 1e-6) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak}
-    traffic = args.traffic if args.traffic is not None else profiled_traffic(dom)
-    roof.update({"kernel": dom, "peak_source": peak_kind + " (MEASURED_PEAKS.json)"
-                 if peak_kind == "measured" else "fallback", "traffic": traffic})
+    cand_host = dw.cand.cpu().numpy() if dw.cand is not None else None
+    accs = []
+    for l, mode in enumerate(w.modes):
+        pooled, emit = _mode_flags(w, mode)
+        accs.append(layer_accounting(w, mode, nvalid, dw.topk_per_layer[l].cpu().numpy(),
+                                     cand_host, pooled=pooled, emit_pool=emit))
+    step_bytes = sum(a["metric"] for a in accs)
 
-    # ---- end to end through the C ABI with pinned host buffers
-    g16 = g16_attention(args, w, dw, csa2, torch, flush_l2, stream, ws, ab, hbm_peak)
+    # ---- per kernel: the first layer's kernels through the individual calls, L2
+    # flushed before each (the scorer and the top-K run back to back, as in a step)
+    peaks = measured_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    kern_us = per_kernel_times(args, w, dw, csa2, torch, flush_l2, stream)
+    acc0 = accs[0]
+    rl = {k: roofline(k, acc0, kern_us[k], peaks, fp8_peak)
+          for k in ("score", "topk", "attn") if k in kern_us and acc0[k] > 0}
+    dom = max(rl, key=lambda k: kern_us[k])
+    roof = dict(rl[dom])
+    units = acc0["selected"] if dom == "attn" else acc0["keys"]
+    traffic, traffic_note = profiled_traffic(dom, w.name, units)
+    roof.update({"peak_source": peaks["source"] + (" x %.0f (nominal FP8/bf16)" % FP8_OVER_BF16
+                                                  if roof["bound"] == "tensor" and dom == "score"
+                                                  else ""),
+                 "traffic": traffic, "traffic_source": traffic_note})
 
-    e2e = run_e2e(args, w, dw, flush, csa2, torch)
-
-    step_gbs = ab["step"] / (ms_per_step * 1e-3) / 1e9
-    launches_per_step = 3 + (1 if nsplit_ws > 0 else 0)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Tq": w.Tq, "N": w.N, "D": w.D, "Hq": w.Hq,
-                   "Hi": w.Hi, "Di": w.Di, "K": w.K, "context_tokens": 4 * w.N,
+                   "Hi": w.Hi, "Di": w.Di, "K": w.K, "C": w.C, "modes": list(w.modes),
+                   "context_tokens": 4 * w.N,
                    "kv_format": "E2M1 + E4M3 scale per channel per 64 entries",
-                   "arith": "indexer e4m3 x e4m3 -> f32; attention f16 x f16 -> f32; out bf16",
                    "l2": "flushed between timed steps (256 MiB write, then a 256 MiB read so the "
                          "flush's dirty lines are written back outside the timed events)",
                    "parallelism": "dp%d (independent batches per GPU)" % world},
-        "step_algorithmic_bytes": ab["step"],
-        "step_gbs": step_gbs, "step_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
-        "step_frac_of_measured_hbm": step_gbs / hbm_peak,
-        "query_tokens_per_s": value * w.B * w.Tq,
-        "kernel_us": kern_us,
-        "roofline": roof,
-        "attn_kv_g16": g16,
-        "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "step_algorithmic_bytes": step_bytes,
+        "step_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
     }
+    line["step_frac_of_8tbs"] = line["step_gbs"] / NOMINAL_HBM_GBS
+    line["step_frac_of_measured_hbm"] = line["step_gbs"] / peaks["hbm_gbs"]
+    line["query_tokens_per_s"] = value * w.B * w.Tq
+    line["per_layer"] = [{"mode": m, "us": 1e3 * statistics.mean(layer_ms[l]),
+                          "algorithmic_bytes": accs[l]["metric"],
+                          "gbs": accs[l]["metric"] / (statistics.mean(layer_ms[l]) * 1e-3) / 1e9}
+                         for l, m in enumerate(w.modes)]
+    line["kernel_us"] = kern_us
+    line["roofline"] = roof
+    line["kernel_rooflines"] = {k: {kk: v[kk] for kk in ("bound", "achieved", "unit", "frac",
+                                                         "hbm_frac")}
+                                for k, v in rl.items()}
+    if w.name == DEFAULT_WORKLOAD:
+        line["attn_kv_g16"] = g16_attention(args, w, dw, csa2, torch, flush_l2, stream, acc0,
+                                            peaks)
+        if not args.no_prefill:
+            line["prefill_indexer"] = prefill_indexer(args, dev, csa2, torch, flush_l2, stream,
+                                                      peaks)
+    if w.name == "prefill_chunk_4096_full":
+        line["prefill_indexer"] = indexer_vs_fp8(kern_us["score"], acc0, peaks, dev)
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, w, dw, csa2, torch)
+    launches = sum({"FULL": 3, "REINDEX": 3, "REUSE": 1}[m] for m in w.modes)
+    launches += sum(2 for m in w.modes if m == "FULL" and w.C and w.pool_block == 8)
+    line["gpu_launches"] = launches * args.steps
+    line["clocks"] = clk.summary()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample_rows)
     if world > 1:
@@ -331,7 +455,107 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def g16_attention(args, w, dw, csa2, torch, flush_l2, stream, ws, ab, hbm_peak):
+def per_kernel_times(args, w, dw, csa2, torch, flush_l2, stream) -> dict:
+    """Device time of each kernel of the workload's first layer, called one by
+    one (events between them), averaged over the timed iterations."""
+    mode = w.modes[0]
+    dev = dw.idx_k.device
+    out = torch.empty_like(dw.out[0])
+    lse = torch.empty_like(dw.lse[0])
+    ws_attn = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K)
+    ws = torch.empty(max(int(ws_attn), 256), dtype=torch.uint8, device=dev)
+    scores = torch.empty((w.B, w.Tq, w.N), dtype=torch.float32, device=dev) \
+        if mode != "REUSE" else None
+    topk = torch.empty_like(dw.topk)
+    kern = {"score": [], "topk": [], "attn": []}
+    if w.name == DEFAULT_WORKLOAD:
+        kern["block_pool"] = []
+        pool_out = torch.empty((w.B, w.Tq, 2048 * 8), dtype=torch.int32, device=dev)
+        pool_ws = torch.empty(max(int(csa2.load().csa2_block_pool_workspace_bytes(
+            w.B, w.Tq, w.N, 8, 2048)), 256), dtype=torch.uint8, device=dev)
+    for i in range(args.warmup + args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        if mode != "REUSE":
+            flush_l2(i)
+            e[0].record(stream)
+            csa2.csa2_index_score(dw.idx_q[0], dw.idx_w[0], dw.idx_k, nvalid=dw.nvalid,
+                                  out=scores)
+            e[1].record(stream)
+            csa2.csa2_topk(scores, w.K, nvalid=dw.nvalid, out=topk)
+            e[2].record(stream)
+            if "block_pool" in kern:
+                csa2.csa2_block_pool(scores, dw.nvalid, 2048, 8, out=pool_out, workspace=pool_ws)
+                e[3].record(stream)
+        else:
+            topk.copy_(dw.topk)
+        flush_l2(i)
+        e[4].record(stream)
+        csa2.csa2_sparse_attn(dw.q[0], dw.kv_packed, dw.kv_scale, topk, w.softmax_scale,
+                              out=out, lse=lse, workspace=ws)
+        e[5].record(stream)
+        torch.cuda.synchronize()
+        if i < args.warmup:
+            continue
+        if mode != "REUSE":
+            kern["score"].append(e[0].elapsed_time(e[1]))
+            kern["topk"].append(e[1].elapsed_time(e[2]))
+            if "block_pool" in kern:
+                kern["block_pool"].append(e[2].elapsed_time(e[3]))
+        kern["attn"].append(e[4].elapsed_time(e[5]))
+    csa2.check_device_errors()
+    return {k: 1e3 * statistics.mean(v) for k, v in kern.items() if v}
+
+
+def indexer_vs_fp8(score_us: float, acc: dict, peaks: dict, dev) -> dict:
+    flops = acc["score_flops"]
+    ach = flops / (score_us * 1e-6) / 1e12
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    r = {"kernel": "index_score_tc_kernel", "us": score_us, "flops": flops,
+         "achieved_tflops": ach, "peak_tflops": fp8_peak,
+         "peak_source": peaks["source"] + " bf16 x %.0f (nominal FP8/bf16)" % FP8_OVER_BF16,
+         "frac": ach / fp8_peak,
+         "flops_rule": "2 x Hi x Di per visible (query, entry) pair"}
+    try:
+        live = fp8_matmul_peak_live(dev)
+        r["fp8_gemm_tflops_live"] = live
+        r["frac_of_live_fp8_gemm"] = ach / live
+        r["live_source"] = "torch._scaled_mm E4M3 8192^3 -> bf16, best of 10, this run"
+    except Exception as ex:   # the live figure is context only
+        r["fp8_gemm_tflops_live"] = None
+        r["live_source"] = "unavailable: %s" % type(ex).__name__
+    return r
+
+
+def prefill_indexer(args, dev, csa2, torch, flush_l2, stream, peaks) -> dict:
+    """The 4096-query prefill chunk's indexer alone (a dense E4M3 contraction of
+    4096 x 65536 x 128 per head, causally masked), timed like the step kernels."""
+    from fp4_kv_cache_step_b200 import workloads as wl
+    w = wl.PREFILL_CHUNK
+    idx_k = torch.from_numpy(wl.idx_k(w)).to(dev)
+    idx_q = torch.from_numpy(wl.idx_q(w, 0)).to(dev)
+    idx_w = torch.from_numpy(wl.idx_w(w, 0)).to(dev)
+    nv = wl.nvalid(w)
+    nvalid = torch.from_numpy(nv).to(dev)
+    scores = torch.empty((w.B, w.Tq, w.N), dtype=torch.float32, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush_l2(i)
+        e0.record(stream)
+        csa2.csa2_index_score(idx_q, idx_w, idx_k, nvalid=nvalid, out=scores)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    csa2.check_device_errors()
+    acc = {"score_flops": int(np.minimum(nv, w.N).astype(np.int64).sum()) * w.Hi * w.Di * 2}
+    r = indexer_vs_fp8(1e3 * statistics.mean(times), acc, peaks, dev)
+    r["workload"] = w.name
+    del scores
+    return r
+
+
+def g16_attention(args, w, dw, csa2, torch, flush_l2, stream, acc, peaks):
     """The attention kernel over the pages' own FP4 layout (one E4M3 scale per
     16 channels of an entry, 288-byte rows): the step's cache dequantised and
     re-quantised into that layout, the same queries and top-K, timed like the
@@ -341,6 +565,8 @@ def g16_attention(args, w, dw, csa2, torch, flush_l2, stream, ws, ab, hbm_peak):
     del kv
     out = torch.empty_like(dw.out[0])
     lse = torch.empty_like(dw.lse[0])
+    need = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K)
+    ws = torch.empty(max(int(need), 256), dtype=torch.uint8, device=rows.device)
     times = []
     for i in range(args.warmup + args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -354,145 +580,259 @@ def g16_attention(args, w, dw, csa2, torch, flush_l2, stream, ws, ab, hbm_peak):
             times.append(e0.elapsed_time(e1))
     csa2.check_device_errors()
     us = 1e3 * statistics.mean(times)
-    gbs = ab["attn_g16"] / (us * 1e-6) / 1e9
+    rows_q = w.B * w.Tq
+    byts = acc["selected"] * (w.D // 2 + w.D // 16) + 2 * rows_q * w.Hq * w.D * 2 + rows_q * w.K * 4
+    gbs = byts / (us * 1e-6) / 1e9
     return {"layout": "E2M1 + E4M3 scale per 16 channels of an entry (288 B rows)",
-            "attn_us": us, "algorithmic_bytes": ab["attn_g16"], "gbs": gbs,
-            "frac_of_measured_hbm": gbs / hbm_peak,
+            "attn_us": us, "algorithmic_bytes": byts, "gbs": gbs,
+            "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
             "cache": "the step's block-scaled cache dequantised and re-quantised per 16 channels"}
 
 
-def run_e2e(args, w, dw, flush, csa2, torch):
-    """The metric through the public call, end to end: every step copies its
-    query-side inputs (queries, indexer queries and weights, lengths) from pinned
-    host memory, runs csa2_layer_step, and copies the attention output and lse
-    back to pinned host memory. The FP4 cache and the indexer keys stay resident
-    (they are the cache). Steps are issued round-robin on three streams with their
-    own buffers and their own copy of the cache, as a serving loop over several
-    sequences' caches would, so one step's copies overlap another's kernels; the
-    value is steps / elapsed device time from the first timed step's start to the
-    last one's end."""
+def run_e2e(args, w, dw, csa2, torch):
+    """The metric through the public call, end to end, one step after another on
+    one stream: every step copies its query-side inputs (attention queries,
+    indexer queries and weights of every layer, lengths) from pinned host memory,
+    runs the workload's layers with csa2_layer_step, and copies every layer's
+    attention output and lse back to pinned host memory. The FP4 cache and the
+    indexer keys stay resident (they are the cache); consecutive steps read
+    three different copies of it in turn, so no step finds the previous step's
+    data in L2. value = steps / device time from the first timed step's start to
+    the last one's end."""
     from fp4_kv_cache_step_b200 import workloads as wl
     nslot = 3
     dev = dw.idx_k.device
-    host_in = {
-        "q": torch.from_numpy(wl.q(w, 0).view(np.int16)).view(torch.bfloat16).pin_memory(),
-        "idx_q": torch.from_numpy(wl.idx_q(w, 0)).pin_memory(),
-        "idx_w": torch.from_numpy(wl.idx_w(w, 0)).pin_memory(),
-        "nvalid": torch.from_numpy(wl.nvalid(w)).pin_memory(),
-    }
+    host_in = {"nvalid": torch.from_numpy(wl.nvalid(w)).pin_memory()}
+    for l, mode in enumerate(w.modes):
+        host_in["q%d" % l] = torch.from_numpy(wl.q(w, l).view(np.int16)).view(
+            torch.bfloat16).pin_memory()
+        if mode != "REUSE":
+            host_in["idx_q%d" % l] = torch.from_numpy(wl.idx_q(w, l)).pin_memory()
+            host_in["idx_w%d" % l] = torch.from_numpy(wl.idx_w(w, l)).pin_memory()
     slots = []
     for si in range(nslot):
         d = {k: torch.empty_like(t, device=dev) for k, t in host_in.items()}
-        # each slot attends over its own copy of the cache, so consecutive steps
-        # stream different 100 MB key sets and L2 cannot carry one into the next
         kvp = dw.kv_packed if si == 0 else dw.kv_packed.clone()
         kvs = dw.kv_scale if si == 0 else dw.kv_scale.clone()
         ik = dw.idx_k if si == 0 else dw.idx_k.clone()
         d["topk"] = torch.full_like(dw.topk, -1)
-        d["out"] = torch.empty_like(dw.out[0])
-        d["lse"] = torch.empty_like(dw.lse[0])
-        d["host_out"] = torch.empty(d["out"].shape, dtype=torch.bfloat16).pin_memory()
-        d["host_lse"] = torch.empty(d["lse"].shape, dtype=torch.float32).pin_memory()
-        d["shared"] = csa2.Csa2Shared(kvp, kvs, ik, d["topk"], None)
-        d["args"] = csa2.layer_args(d["q"], d["nvalid"], d["out"], w.K, w.softmax_scale,
-                                    idx_q=d["idx_q"], idx_w=d["idx_w"], lse=d["lse"], N=w.N)
-        need = csa2.layer_step_workspace_bytes(wl.FULL, d["args"], d["shared"])
-        d["ws"] = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-        d["stream"] = torch.cuda.Stream(device=dev)
+        d["cand"] = torch.full_like(dw.cand, -1) if dw.cand is not None else None
+        d["shared"] = csa2.Csa2Shared(kvp, kvs, ik, d["topk"], d["cand"])
+        d["out"], d["lse"], d["host_out"], d["host_lse"], d["args"] = [], [], [], [], []
+        need = 256
+        for l, mode in enumerate(w.modes):
+            o = torch.empty_like(dw.out[l])
+            ls = torch.empty_like(dw.lse[l])
+            d["out"].append(o)
+            d["lse"].append(ls)
+            d["host_out"].append(torch.empty(o.shape, dtype=torch.bfloat16).pin_memory())
+            d["host_lse"].append(torch.empty(ls.shape, dtype=torch.float32).pin_memory())
+            pooled, emit = _mode_flags(w, mode)
+            a = csa2.layer_args(d["q%d" % l], d["nvalid"], o, w.K, w.softmax_scale,
+                                idx_q=d.get("idx_q%d" % l), idx_w=d.get("idx_w%d" % l), lse=ls,
+                                N=w.N, emit_pool=(0 if not emit else (2 if w.pool_block == 8
+                                                                      else 1)),
+                                use_pool=pooled)
+            d["args"].append(a)
+            need = max(need, csa2.layer_step_workspace_bytes(mode, a, d["shared"]))
+        d["ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
         slots.append(d)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = slots[0]["host_out"].numel() * 2 + slots[0]["host_lse"].numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in slots[0]["host_out"] + slots[0]["host_lse"])
 
     def one_step(d):
-        with torch.cuda.stream(d["stream"]):
-            for k, t in host_in.items():
-                d[k].copy_(t, non_blocking=True)
-            csa2.csa2_layer_step(wl.FULL, d["args"], d["shared"], d["ws"])
-            d["host_out"].copy_(d["out"], non_blocking=True)
-            d["host_lse"].copy_(d["lse"], non_blocking=True)
+        for k, t in host_in.items():
+            d[k].copy_(t, non_blocking=True)
+        for l, mode in enumerate(w.modes):
+            csa2.csa2_layer_step(mode, d["args"][l], d["shared"], d["ws"])
+        for l in range(len(w.modes)):
+            d["host_out"][l].copy_(d["out"][l], non_blocking=True)
+            d["host_lse"][l].copy_(d["lse"][l], non_blocking=True)
 
+    stream = torch.cuda.current_stream()
     for i in range(args.warmup):
         one_step(slots[i % nslot])
     torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    start.record(torch.cuda.current_stream())
-    for d in slots:
-        d["stream"].wait_event(start)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
     for i in range(args.steps):
         one_step(slots[i % nslot])
-    ends = []
-    for d in slots:
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(d["stream"])
-        ends.append(e)
+    end.record(stream)
     torch.cuda.synchronize()
-    ms = max(start.elapsed_time(e) for e in ends) / args.steps
-    return {"value": 1e3 / ms, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "streams": nslot,
-            "l2": "not flushed: the three slots' caches (3 x 410 MB) are read in turn, so "
-                  "no step finds the previous step's keys in L2"}
+    csa2.check_device_errors()
+    ms = start.elapsed_time(end) / args.steps
+    _, unit = workload_metric(w)
+    return {"value": 1e3 / ms, "unit": unit, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "streams": 1,
+            "l2": "not flushed: three copies of the cache are read in turn"}
 
 
 # --------------------------------------------------------------- CPU oracle
-def oracle_layer_steps(w, rows):
-    """Time the oracle's FULL layer step on the given batch rows (cache build
-    excluded). Returns seconds."""
-    import oracle
-    from fp4_kv_cache_step_b200 import workloads as wl
-    nv_all = wl.nvalid(w)
-    total = 0.0
-    for b in rows:
-        packed, sc = oracle.fp4_kv_pack(wl.kv(w, rows=[b]))
-        ik = wl.idx_k(w, rows=[b])
-        q = wl.q(w, 0, rows=[b])
-        iq = wl.idx_q(w, 0, rows=[b])
-        iw = wl.idx_w(w, 0, rows=[b])
-        topk = np.full((1, w.Tq, w.K), -1, np.int32)
+def cpu_info():
+    model = platform.processor() or "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count() or 1
+
+
+def oracle_units(w, n: int):
+    """Independent units of work of a workload for the oracle: (batch row, first
+    query, end query). Decode workloads: whole sequences (one query each). The
+    prefill chunk (one sequence of 4096 queries): single queries, n of them
+    spread evenly over the chunk."""
+    if w.Tq == 1:
+        return [(b, 0, 1) for b in range(min(n, w.B))]
+    n = max(1, min(n, w.B * w.Tq))
+    step = w.B * w.Tq / n
+    out = []
+    for i in range(n):
+        r = int(i * step)
+        out.append((r // w.Tq, r % w.Tq, r % w.Tq + 1))
+    return out
+
+
+class OracleSequences:
+    """The oracle's inputs for some units of a workload (see oracle_units; the
+    FP4 cache packed by the oracle itself), prepared once; `step(units, threads)`
+    runs the workload's mode schedule on them, one thread per unit (each unit is
+    an independent problem; the oracle's calls release the interpreter lock)."""
+
+    def __init__(self, w, units, threads):
+        import oracle
+        from fp4_kv_cache_step_b200 import workloads as wl
+        oracle.build()
+        self.w, self.oracle = w, oracle
+        nv_all = wl.nvalid(w)
+        # one small call first, on this thread (the oracle fills its E4M3 table once)
+        oracle.fp4_kv_pack(np.zeros((1, 64, 64), np.float32))
+        oracle.index_score(np.zeros((1, 1, 1, 16), np.uint8), np.ones((1, 1, 1), np.float32),
+                           np.zeros((1, 64, 16), np.uint8), nvalid=np.full((1, 1), 64, np.int32))
+        cache = {}
+
+        def seq(b):
+            if b not in cache:
+                packed, sc = oracle.fp4_kv_pack(wl.kv(w, rows=[b]))
+                cache[b] = (packed, sc, wl.idx_k(w, rows=[b]),
+                            [(mode, wl.q(w, l, rows=[b]),
+                              wl.idx_q(w, l, rows=[b]) if mode != "REUSE" else None,
+                              wl.idx_w(w, l, rows=[b]) if mode != "REUSE" else None)
+                             for l, mode in enumerate(w.modes)])
+            return cache[b]
+
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(seq, sorted({u[0] for u in units})))
+
+        def part(a, t0, t1):
+            return None if a is None else np.ascontiguousarray(a[:, t0:t1])
+        self.data = {}
+        for (b, t0, t1) in units:
+            packed, sc, ik, layers = cache[b]
+            self.data[(b, t0, t1)] = {
+                "packed": packed, "scale": sc, "idx_k": ik,
+                "nvalid": np.ascontiguousarray(nv_all[b:b + 1, t0:t1]),
+                "layers": [(m, part(q, t0, t1), part(iq, t0, t1), part(iw, t0, t1))
+                           for m, q, iq, iw in layers]}
+
+    def _one(self, u):
+        o, w, d = self.oracle, self.w, self.data[u]
+        tq = u[2] - u[1]
+        topk = np.full((1, tq, w.K), -1, np.int32)
+        cand = np.full((1, tq, w.C), -1, np.int32) if w.C else None
+        modes = {"FULL": o.MODE_FULL, "REINDEX": o.MODE_REINDEX, "REUSE": o.MODE_REUSE}
+        for mode, q, iq, iw in d["layers"]:
+            pooled, _ = _mode_flags(w, mode)
+            o.layer_step(modes[mode], q, iq, iw, d["idx_k"], d["packed"], d["scale"],
+                         d["nvalid"], w.K, w.softmax_scale, topk, cand, w.C, use_pool=pooled)
+
+    def step(self, units, threads) -> float:
+        """Seconds for the given units, `threads` at a time."""
         t0 = time.perf_counter()
-        oracle.layer_step(oracle.MODE_FULL, q, iq, iw, ik, packed, sc, nv_all[b:b + 1], w.K,
-                          w.softmax_scale, topk)
-        total += time.perf_counter() - t0
-    return total
+        if threads <= 1:
+            for u in units:
+                self._one(u)
+        else:
+            with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+                list(ex.map(self._one, units))
+        return time.perf_counter() - t0
 
 
 def cpu_baseline(w, nrows):
-    import oracle
-    oracle.build()
-    rows = list(range(min(nrows, w.B)))
-    secs = oracle_layer_steps(w, rows)
-    per_step = secs * w.B / len(rows)
-    return {"value": 1.0 / per_step, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d of %d sequences of one FULL layer step (score + top-K + attention, "
-                      "cache build excluded), single-threaded fp64; scaled to a %d-sequence "
-                      "layer step" % (len(rows), w.B, w.B)}
+    """The oracle on the host cores: one thread on a sample of units, and one
+    thread per unit over every core on the whole batch (or, for the largest
+    workloads, as many units as there are cores), scaled to one step of the
+    workload."""
+    model, ncores = cpu_info()
+    total = w.B * w.Tq
+    big = w.name in ("prefill_chunk_4096_full", "hier_1m_full_pool_reindex")
+    units_mt = oracle_units(w, min(total, ncores) if big else total)
+    units_1 = units_mt[:max(1, min(nrows, len(units_mt)))]
+    data = OracleSequences(w, units_mt, ncores)
+    secs1 = data.step(units_1, 1)
+    per_step1 = secs1 * total / len(units_1)
+    threads = min(ncores, len(units_mt))
+    secs_mt = data.step(units_mt, threads)
+    per_step_mt = secs_mt * total / len(units_mt)
+    _, unit = workload_metric(w)
+    what = "queries" if w.Tq > 1 else "sequences"
+    return {"value": 1.0 / per_step_mt, "unit": unit, "cores": threads, "kind": "oracle",
+            "cpu_model": model, "host_cores": ncores,
+            "sample": "%d of %d %s of one step of the workload's layers (cache build "
+                      "excluded), fp64, one thread per unit on %d threads; scaled to the "
+                      "whole step" % (len(units_mt), total, what, threads),
+            "single_thread": {"value": 1.0 / per_step1, "cores": 1,
+                              "sample": "%d of %d %s, one thread, scaled to the whole step"
+                                        % (len(units_1), total, what)}}
 
 
 def run_reference(args):
+    """The oracle as the reference arm: every step is one whole step of the
+    workload (all its sequences, one thread per sequence over the host's cores)
+    when the host has the cores for it to end within about a second, else as
+    many units as there are cores, scaled to the batch; ms_per_step is the
+    measured time of what each step ran."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    sys.path.insert(0, ROOT)
     from fp4_kv_cache_step_b200 import workloads as wl
-    import oracle
-    oracle.build()
-    w = wl.WORKLOADS[args.workload]
-    for i in range(args.warmup):
-        oracle_layer_steps(w, [i % w.B])
-    secs = [oracle_layer_steps(w, [i % w.B]) for i in range(args.steps)]
-    per_step = statistics.mean(secs) * w.B
-    value = 1.0 / per_step
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "Tq": w.Tq, "N": w.N, "D": w.D, "Hq": w.Hq,
-                       "Hi": w.Hi, "Di": w.Di, "K": w.K, "context_tokens": 4 * w.N,
-                       "parallelism": "none (CPU oracle, rank 0)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": "each step: one sequence of the %d-sequence FULL layer "
-                                       "step, scaled by %d; single-threaded fp64" % (w.B, w.B)},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+    name = getattr(args, "workload", DEFAULT_WORKLOAD)
+    w = wl.WORKLOADS[name]
+    metric, unit = workload_metric(w)
+    model, ncores = cpu_info()
+    total = w.B * w.Tq
+    big = w.name in ("prefill_chunk_4096_full", "hier_1m_full_pool_reindex")
+    n_units = min(total, ncores) if (big or ncores < total // 2) else total
+    units = oracle_units(w, n_units)
+    threads = min(ncores, len(units))
+    data = OracleSequences(w, units, threads)
+    for _ in range(args.warmup):
+        data.step(units, threads)
+    secs = [data.step(units, threads) for _ in range(args.steps)]
+    step_s = statistics.mean(secs)
+    value = len(units) / total / step_s
+    what = "queries" if w.Tq > 1 else "sequences"
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "Tq": w.Tq, "N": w.N, "D": w.D,
+                       "Hq": w.Hq, "Hi": w.Hi, "Di": w.Di, "K": w.K, "C": w.C,
+                       "modes": list(w.modes), "context_tokens": 4 * w.N,
+                       "parallelism": "CPU oracle on rank 0, one thread per %s" % what[:-1]},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                             "cpu_model": model, "host_cores": ncores,
+                             "sample": "each step: %d of %d %s of the workload's step, fp64, "
+                                       "%d threads; ms_per_step is that measured time"
+                                       % (len(units), total, what, threads)},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    if len(units) != total:
+        line["scaled_from"] = "%d of %d %s per step" % (len(units), total, what)
     print(json.dumps(line), flush=True)
 
 
@@ -514,8 +854,7 @@ def run_stack(args):
     st = wl.production_stack(args.context, args.batch)
     ds = DeviceStack(st, dev)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    flush_l2 = L2Flush(torch, dev)
     for _ in range(args.warmup):
         ds.step()
     torch.cuda.synchronize()
@@ -524,8 +863,7 @@ def run_stack(args):
           for _ in range(args.steps)]
     with ClockSampler(dev.index) as clk:
         for i in range(args.steps):
-            flush.fill_(i & 0xff)
-            flush_rd.max()
+            flush_l2(i)
             ev[i][0].record(stream)
             ds.step()
             ev[i][1].record(stream)
@@ -536,12 +874,12 @@ def run_stack(args):
     nlayers = len(st.layers)
     modes = [st.segments[s].modes[l] for s, l in st.layers]
     launches = sum({"FULL": 3, "REINDEX": 3, "REUSE": 1}[m] for m in modes)
-    launches += 3                                      # the decoder FULL's blockwise pool
+    launches += 2                                      # the decoder FULL's blockwise pool
     print(json.dumps({
         "metric": "CSA2 stack decode steps/s (the model's 38 CSA2 layers)",
         "value": 1e3 / ms_per_step, "unit": "stack-steps/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": "production_stack", "context_tokens": args.context,
                    "B": args.batch, "csa2_layers": nlayers, "swa_only_layers": st.swa_only,
                    "encoder_entries": args.context // 2, "decoder_entries": args.context,
@@ -559,16 +897,17 @@ def run_stack(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="workload name (fp4_kv_cache_step_b200.workloads.WORKLOADS)")
-    ap.add_argument("--cpu-sample-rows", type=int, default=8)
+    ap.add_argument("--cpu-sample-rows", type=int, default=4,
+                    help="sequences in the single-threaded oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--attn-bound", default="tensor", choices=["tensor", "hbm"])
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the dominant kernel, if captured")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill-chunk indexer figure of the default line")
     ap.add_argument("--stack", default=None, choices=["production"],
                     help="time the model's 38 CSA2 layers (one GPU) instead of the headline step")
     ap.add_argument("--context", type=int, default=131072, help="--stack: context in tokens")

@@ -43,11 +43,13 @@ csa2_status ok() {
   return CSA2_OK;
 }
 
-int* device_error_word(cudaError_t* e_out) {
+// Enters the stream's device and returns its error word (looked up once per
+// device, with that device current).
+int* device_error_word(cudaStream_t stream, csa2::DeviceScope& scope, cudaError_t* e_out) {
   static std::mutex mu;
   static int* words[128] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = scope.enter(stream);
+  const int dev = scope.device();
   if (e != cudaSuccess || dev < 0 || dev >= 128) {
     *e_out = e != cudaSuccess ? e : cudaErrorInvalidDevice;
     return nullptr;
@@ -168,7 +170,9 @@ csa2_status api_check_attn_args(const uint16_t* q, const uint8_t* kv_packed,
                                 int Hq, int D, int N, int K, const uint16_t* out, const float* lse) {
   return check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
 }
-int* api_error_word(cudaError_t* e) { return device_error_word(e); }
+int* api_error_word(cudaStream_t stream, DeviceScope& scope, cudaError_t* e) {
+  return device_error_word(stream, scope, e);
+}
 csa2_status api_fail(csa2_status s, const char* msg) { return fail(s, "%s", msg); }
 csa2_status api_cuda_fail(cudaError_t e, const char* where) { return cuda_fail(e, where); }
 csa2_status api_ok() { return ok(); }
@@ -182,7 +186,8 @@ csa2_status fp4_kv_pack(const float* kv, int B, int N, int D, uint8_t* kv_packed
   csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
   if (s != CSA2_OK) return s;
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "fp4_kv_pack");
   e = csa2::launch_fp4_pack(kv, B, N, D, kv_packed, kv_scale, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_pack launch");
@@ -194,7 +199,10 @@ csa2_status fp4_kv_unpack(const uint8_t* kv_packed, const uint8_t* kv_scale, int
   CHECK_PTR(out);
   csa2_status s = check_kv(kv_packed, kv_scale, B, N, D);
   if (s != CSA2_OK) return s;
-  cudaError_t e = csa2::launch_fp4_unpack(kv_packed, kv_scale, B, N, D, out, (cudaStream_t)stream);
+  csa2::DeviceScope scope;
+  cudaError_t e = scope.enter((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack device");
+  e = csa2::launch_fp4_unpack(kv_packed, kv_scale, B, N, D, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack launch");
   return ok();
 }
@@ -205,7 +213,8 @@ csa2_status fp4_kv_pack_g16(const float* kv, int B, int N, int D, uint8_t* kv_ro
   csa2_status s = check_kv_g16(kv_rows, B, N, D);
   if (s != CSA2_OK) return s;
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "fp4_kv_pack_g16");
   e = csa2::launch_fp4_pack_g16(kv, nullptr, B, N, N, D, kv_rows, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_pack_g16 launch");
@@ -217,7 +226,10 @@ csa2_status fp4_kv_unpack_g16(const uint8_t* kv_rows, int B, int N, int D, float
   CHECK_PTR(out);
   csa2_status s = check_kv_g16(kv_rows, B, N, D);
   if (s != CSA2_OK) return s;
-  cudaError_t e = csa2::launch_fp4_unpack_g16(kv_rows, B, N, D, out, (cudaStream_t)stream);
+  csa2::DeviceScope scope;
+  cudaError_t e = scope.enter((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack_g16 device");
+  e = csa2::launch_fp4_unpack_g16(kv_rows, B, N, D, out, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_unpack_g16 launch");
   return ok();
 }
@@ -230,7 +242,8 @@ csa2_status fp4_kv_append_g16(const float* kv_new, const int32_t* pos, int B, in
   csa2_status s = check_kv_g16(kv_rows, B, N, D);
   if (s != CSA2_OK) return s;
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "fp4_kv_append_g16");
   e = csa2::launch_fp4_pack_g16(kv_new, pos, B, T, N, D, kv_rows, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_kv_append_g16 launch");
@@ -244,7 +257,8 @@ csa2_status csa2_index_score(const uint8_t* idx_q, const float* idx_w, const uin
   csa2_status s = check_score_args(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid, cand, C);
   if (s != CSA2_OK) return s;
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_index_score");
   e = csa2::launch_index_score(idx_q, idx_w, idx_k, B, Tq, N, Hi, Di, nvalid, cand, cand ? C : 0,
                                scores, err, (cudaStream_t)stream);
@@ -266,7 +280,8 @@ csa2_status csa2_topk(const float* scores, int ld, const int32_t* nvalid, const 
     CHECK_ARG(Cout >= 1 && Cout <= 65536, "Cout=%d must be in [1, 65536]", Cout);
   }
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_topk");
   e = csa2::launch_topk(scores, ld, cand ? nullptr : nvalid, cand, B * Tq, K, topk_idx,
                         cand_out ? Cout : 0, cand_out, err, (cudaStream_t)stream);
@@ -291,7 +306,8 @@ csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const 
     return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn needs %zu workspace bytes (got %zu)", need,
                 workspace_bytes);
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_sparse_attn");
   e = csa2::launch_sparse_attn(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, N, K, softmax_scale,
                                out, lse, workspace, err, (cudaStream_t)stream);
@@ -310,7 +326,8 @@ csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows,
     return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn_g16 needs %zu workspace bytes (got %zu)",
                 need, workspace_bytes);
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_sparse_attn_g16");
   // a NULL block-scale array selects the 16-channel layout
   e = csa2::launch_sparse_attn(q, kv_rows, nullptr, topk_idx, B, Tq, Hq, N, K, softmax_scale, out,
@@ -340,7 +357,8 @@ csa2_status csa2_block_pool(const float* scores, int ld, const int32_t* nvalid, 
     return fail(CSA2_ERR_WORKSPACE, "csa2_block_pool needs %zu workspace bytes (got %zu)", need,
                 workspace_bytes);
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_block_pool");
   e = csa2::launch_block_pool(scores, ld, nvalid, B * Tq, block, nblocks, cand_out, workspace, err,
                               (cudaStream_t)stream);
@@ -398,7 +416,8 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
     return fail(CSA2_ERR_WORKSPACE, "csa2_layer_step needs %zu workspace bytes (got %zu)", need,
                 workspace_bytes);
   cudaError_t e;
-  int* err = device_error_word(&e);
+  csa2::DeviceScope scope;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_layer_step");
   cudaStream_t cs = (cudaStream_t)stream;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -430,7 +449,10 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
 }
 
 csa2_status csa2_check_device_errors(csa2_stream_t stream) {
-  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  csa2::DeviceScope scope;   // the error word of the stream's device
+  cudaError_t e = scope.enter((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_check_device_errors device");
+  e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "csa2_check_device_errors sync");
   int code = 0, zero = 0;
   e = cudaMemcpyFromSymbol(&code, g_device_error, sizeof(int));

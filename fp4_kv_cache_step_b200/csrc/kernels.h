@@ -38,12 +38,50 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Makes the device a stream belongs to current for the rest of an entry point
+// (restoring the caller's current device on exit), so that the error word, any
+// built-in scratch and every launch belong to the stream's device. The legacy
+// and per-thread default streams belong to the current device.
+class DeviceScope {
+ public:
+  DeviceScope() = default;
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+  ~DeviceScope() {
+    if (prev_ >= 0) cudaSetDevice(prev_);
+  }
+  cudaError_t enter(cudaStream_t s) {
+    int cur = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    int dev = cur;
+    if (s != nullptr && s != cudaStreamLegacy && s != cudaStreamPerThread) {
+      e = cudaStreamGetDevice(s, &dev);
+      if (e != cudaSuccess) return e;
+    }
+    if (dev != cur) {
+      e = cudaSetDevice(dev);
+      if (e != cudaSuccess) return e;
+      prev_ = cur;
+    }
+    dev_ = dev;
+    return cudaSuccess;
+  }
+  int device() const { return dev_; }
+
+ private:
+  int prev_ = -1;
+  int dev_ = 0;
+};
+
 // Argument checks, error word and last-error text of api.cu, for entry points
 // that live in other files.
 csa2_status api_check_attn_args(const uint16_t* q, const uint8_t* kv_packed,
                                 const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
                                 int Hq, int D, int N, int K, const uint16_t* out, const float* lse);
-int* api_error_word(cudaError_t* e);
+// Enters the stream's device (see DeviceScope) and returns that device's error
+// word, or nullptr with *e set.
+int* api_error_word(cudaStream_t stream, DeviceScope& scope, cudaError_t* e);
 csa2_status api_fail(csa2_status s, const char* msg);
 csa2_status api_cuda_fail(cudaError_t e, const char* where);
 csa2_status api_ok();

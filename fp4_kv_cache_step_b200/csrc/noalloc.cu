@@ -21,7 +21,13 @@
 //    reads it;
 //  - the first call on each device looks up the array's device address (a
 //    host-side symbol query that may load this module), so make that first
-//    call outside any stream capture.
+//    call outside any stream capture;
+//  - the call runs on the device its stream belongs to, which it makes current
+//    for the lookup and the launch (the caller's current device is restored);
+//  - under CUDA's lazy module loading (the default since CUDA 12) the array is
+//    reserved on a device when this module is first used there; with
+//    CUDA_MODULE_LOADING=EAGER every context that loads the library reserves
+//    it, whether or not this entry point is ever called.
 // No cudaMalloc, cudaFree or allocating library routine is called.
 #include <mutex>
 #include <string>
@@ -37,17 +43,16 @@ constexpr size_t kNoAllocScratchBytes = CSA2_NOALLOC_SCRATCH_BYTES;
 // symbol: its device address must be fetched with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device, with that device current).
-void* scratch_address(cudaError_t* e_out) {
+// Device address of g_noalloc_scratch on device `dev`, which must be current
+// (looked up once per device).
+void* scratch_address(int dev, cudaError_t* e_out) {
   static std::mutex mu;
   static void* addr[128] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= 128) {
-    *e_out = e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 128) {
+    *e_out = cudaErrorInvalidDevice;
     return nullptr;
   }
+  cudaError_t e;
   std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
@@ -82,11 +87,12 @@ csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* kv_packed
     return csa2::api_fail(CSA2_ERR_WORKSPACE, msg.c_str());
   }
   cudaError_t e;
-  int* err = csa2::api_error_word(&e);
+  csa2::DeviceScope scope;   // the stream's device is current from here on
+  int* err = csa2::api_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return csa2::api_cuda_fail(e, "csa2_sparse_attn_noalloc");
   void* scratch = nullptr;
   if (need > 0) {
-    scratch = scratch_address(&e);
+    scratch = scratch_address(scope.device(), &e);
     if (!scratch) return csa2::api_cuda_fail(e, "csa2_sparse_attn_noalloc scratch address");
   }
   e = csa2::launch_sparse_attn(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, N, K, softmax_scale,

@@ -21,7 +21,11 @@
  *    The library allocates no device memory; scratch comes from the caller's
  *    workspace (size from the matching *_workspace_bytes query).
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
- *    default stream). Host-side argument errors are reported before anything is
+ *    default stream) and runs on the device that stream belongs to: the call
+ *    makes that device current while it works and restores the caller's
+ *    current device before it returns (the legacy and per-thread default
+ *    streams belong to the current device). Device pointers must be on that
+ *    device. Host-side argument errors are reported before anything is
  *    launched; nothing is thrown across the ABI.
  *  - Device-side data errors (an index outside [-1, N), a non-finite value, an
  *    unsorted candidate list) do not trap: the kernel skips the bad element and
@@ -260,16 +264,20 @@ CSA2_API csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_r
  * no allocator, or a latency-critical path that must avoid an allocation and
  * its implicit synchronisation. Same arguments, semantics and results as
  * csa2_sparse_attn minus the workspace: the split scratch comes from a fixed
- * device array of CSA2_NOALLOC_SCRATCH_BYTES built into the library (resident
- * on every device that called this function, until the process exits).
+ * device array of CSA2_NOALLOC_SCRATCH_BYTES built into the library. Under
+ * CUDA's lazy module loading (the default since CUDA 12) the array is reserved
+ * on a device when this function is first used there and stays until the
+ * process exits; with CUDA_MODULE_LOADING=EAGER every context that loads the
+ * library reserves it, whether or not this function is ever called.
  *  - Returns CSA2_ERR_WORKSPACE, launching nothing, when the shape needs more
  *    split scratch than the array holds (compare with
  *    csa2_sparse_attn_workspace_bytes()).
  *  - All calls on a device share the array: calls that overlap on the GPU
  *    (e.g. two streams at once) race. The array keeps the last call's contents;
  *    nothing in it needs to start at zero.
- *  - The first call on each device looks up the array's address on the host;
- *    make that first call before any stream capture.
+ *  - The first call on each device looks up the array's address on the host
+ *    (with the stream's device current); make that first call before any
+ *    stream capture.
  *  - Calls no cudaMalloc, cudaFree or allocating library routine.
  * ------------------------------------------------------------------------ */
 #define CSA2_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
@@ -330,7 +338,7 @@ CSA2_API csa2_status csa2_layer_step(const csa2_layer_args* args, csa2_mode mode
 /* ------------------------------------------------------------------------
  * Errors.
  * csa2_check_device_errors: synchronises `stream`, returns the first device
- * data error recorded on the current device since the last check (CSA2_OK if
+ * data error recorded on the stream's device since the last check (CSA2_OK if
  * none) and clears it.
  * csa2_last_error: thread-local text for the last non-OK status returned on
  * this thread (empty string if none). The pointer stays valid until the next
