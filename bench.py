@@ -195,9 +195,16 @@ def layer_accounting(w, mode: str, nvalid: np.ndarray, topk: np.ndarray, cand=No
         acc["score"] = keys * (w.Di + 4) + c.size * 4 + idx_qw
         acc["topk"] = keys * 4 + c.size * 4 + idx
     else:
-        keys = int(np.minimum(nvalid.reshape(-1).astype(np.int64), w.N).sum())
-        acc["score"] = keys * (w.Di + 4) + idx_qw
+        nv = np.minimum(nvalid.reshape(w.B, w.Tq).astype(np.int64), w.N)
+        keys = int(nv.sum())                       # (query, visible entry) pairs scored
+        # every query of a sequence scores the same keys: each is read once
+        uniq = int(nv.max(axis=1).sum())
+        acc["score"] = uniq * w.Di + keys * 4 + idx_qw
         acc["topk"] = keys * 4 + idx + (rows * w.C * 4 if emit_pool else 0)
+        acc["metric"] += uniq * w.Di + idx_qw
+        acc["keys"] = keys
+        acc["score_flops"] = keys * w.Hi * w.Di * 2
+        return acc
     acc["keys"] = keys
     acc["score_flops"] = keys * w.Hi * w.Di * 2
     acc["metric"] += keys * w.Di + idx_qw
@@ -290,15 +297,20 @@ class ClockSampler:
 class L2Flush:
     """Writes 256 MiB (evicting every line of the step's data), then reads
     another 256 MiB so that the dirty flush lines are written back here,
-    outside the timed events, not by the next step's first kernel."""
+    outside the timed events, not by the next step's first kernel. Then the
+    GPU spins for about 300 us, so that the host has queued everything the
+    timed region launches before its first event fires (the events then see
+    device time only, no gap while the host is still launching)."""
 
     def __init__(self, torch, dev):
+        self.torch = torch
         self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
 
     def __call__(self, i: int):
         self.w.fill_(i & 0xff)
         self.r.max()
+        self.torch.cuda._sleep(600000)
 
 
 def _mode_flags(w, mode):

@@ -76,6 +76,11 @@ SplitPlan plan_splits(int rows, int Hq, int K) {
   const int ctas = rows * p.nhb;
   const int sms = sm_count();
   int nsplit = ctas >= sms ? 1 : sms / ctas;
+  // up to twice the largest cluster, the splits stay one cluster that merges on
+  // chip (a few idle SMs cost less than the workspace round trip and the
+  // combine launch)
+  const int cmax = sparse_attn_tc_max_cluster();
+  if (nsplit > cmax && nsplit < 2 * cmax) nsplit = cmax;
   nsplit = min(nsplit, ceil_div(K, tile));
   nsplit = max(nsplit, 1);
   p.split_len = ceil_div(ceil_div(K, nsplit), tile) * tile;

@@ -9,27 +9,34 @@
 // which serves as both key and value).
 //
 // One CTA = (query row, block of 64 heads, split of the selected-entry list),
-// processed in tiles of 64 entries through a two-deep pipeline: while the
-// softmax works on tile t, the tensor core runs P(t-1) V(t-1) and S(t+1), and
-// the producers dequantise tile t+2. Every selected row is gathered and
-// dequantised ONCE, into a shared-memory tile that serves both products:
-//   S(t) = Q V(t)^T   M = 64 heads, N = 64 entries, K = 512 (32 MMAs, V tile
-//                     read K-major), accumulator in TMEM lanes 16-31 (two
-//                     buffers of 64 columns);
-//   O   += P(t) V(t)  M = 64 heads, N = 256 dims per half, K = 64 entries
-//                     (8 MMAs, V tile read MN-major), accumulator in TMEM
-//                     lanes 0-15, all 512 columns.
-// A softmax thread owns one head: its 64 logits of a tile, its reference
-// maximum and its row sum live in registers, so the softmax needs no barrier.
-// The maximum is lazy: P = 2^(s - m) with m raised (and O, l rescaled) only
-// when a tile holds a logit more than 8 above it, so P stays below 2^8 in fp16
-// and rescaling is rare.
-// Values are dequantised with integer ops only (E2M1 magnitudes from a byte
-// table, E4M3 scales shifted into fp16 fields); they carry an exact factor 2^-8
-// that the softmax scale and the epilogue undo.
-// Roles: warps 0-7 gather and dequantise; warp 8 owns TMEM and issues the MMAs;
-// warps 9-12 stage Q, run the softmax (S rows in lanes 16-31 of their
-// quadrant), the O rescales and the epilogue (O rows in lanes 0-15). Every
+// processed in tiles of 64 entries through three-deep rings: while the softmax
+// works on tile t, the tensor core runs P(t-1) V(t-1) and S(t+1), and the
+// producers fill tile t+2. Every selected row is gathered and dequantised ONCE,
+// into a shared-memory tile that serves both products:
+//   S(t) = Q V(t)^T   M = 64 heads, N = 64 entries, K = 512: 32 MMAs with the
+//                     query block as the A operand held in tensor memory (so
+//                     only the V tile is read from shared memory) and the V
+//                     tile read K-major;
+//   O   += P(t) V(t)  M = 64 heads, N = 256 dims per half, K = 64 entries:
+//                     8 MMAs, P and the V tile (read MN-major) from shared memory.
+// Tensor memory (an M = 64 operand or accumulator occupies 16 lanes of each
+// 32-lane quadrant): lanes 0-15 hold S(t) (three buffers of 64 columns) and the
+// query block (256 columns of fp16 pairs, columns 192-447); lanes 16-31 hold O
+// (all 512 columns).
+// A softmax thread owns half of one head's 64 logits of a tile (the other half
+// is the thread 16 lanes away): its logits, the head's reference maximum and
+// its part of the row sum live in registers. The maximum is lazy: P = 2^(s - m)
+// with m raised (and O and the row sum rescaled) only when a tile holds a logit
+// more than 8 above it, so P stays below 2^8 in fp16 and rescaling is rare.
+// Values are dequantised with integer ops (E2M1 magnitudes from a byte table,
+// E4M3 scales shifted into fp16 fields); they carry an exact factor 2^-8 that
+// the softmax scale and the epilogue undo. A producer dequantises a tile into
+// registers BEFORE waiting for its ring slot, so after the slot frees only the
+// shared-memory stores stand between P(t-3) V(t-3) and S(t).
+// Roles: warps 0-7 gather and dequantise; warp 8 owns tensor memory and issues
+// the MMAs; warps 9-12 stage Q into tensor memory and run the softmax. At the
+// end every warp that can reach a quadrant's O lanes (its softmax warp and two
+// producer warps) writes that quadrant's output, partial or final. Every
 // mbarrier wait is bounded.
 #include <cooperative_groups.h>
 
@@ -47,33 +54,60 @@ using namespace sm100;
 constexpr int kD = kHeadDim;             // 512
 constexpr int kHB = 64;                  // heads per CTA
 constexpr int kT = 64;                   // entries per tile
-constexpr int kAtom = 8192;              // 64 rows x 128 B: a K atom of Q or P, or of a V tile
+constexpr int kAtom = 8192;              // 64 rows x 128 B: a K atom of P, or of a V tile
 constexpr int kVTile = 8 * kAtom;        // 64 entries x 512 dims of fp16
+constexpr int kRing = 3;                 // V tiles, S buffers and P buffers in flight
 constexpr int kProducerWarps = 8;
 constexpr int kMmaWarp = 8;
 constexpr int kThreads = 13 * 32;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemQ = 192;         // first column of the query block (lanes 0-15)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.0f;    // log2 units: P <= 2^8 before a rescale
+constexpr int kMaxClusterSplits = 8;
 
 struct __align__(8) Bars {
-  uint64_t q_full, o_full;
-  uint64_t v_full[2], v_free[2], s_full[2], p_full[2], p_free[2];
+  uint64_t q_ld, q_conv, q_full, q_free, o_full, recv;
+  uint64_t v_full[kRing], v_free[kRing], s_full[kRing], p_full[kRing];
 };
 
 struct Smem {
   Bars bar;
   uint32_t tmem_slot;
   int abort_flag;
-  uint32_t valid[2][kT / 32];   // bit i of word w: entry 32 w + i of the tile is selected
-                                // (byte w of a buffer written by producer warp w)
-  float head_scale[kHB];
-  float2 ml[kHB];               // this split's (reference maximum, row sum) per head
+  uint32_t valid[kRing][kT / 32];   // bit i of word w: entry 32 w + i of the tile is selected
+                                    // (byte w' of the pair written by producer warp w')
+  float2 mlf[kHB];                  // this split's (reference maximum, row sum) per head
+  float qdown[kHB];                 // the power of two each head's query was scaled up by, inverted
 };
 
-constexpr size_t kSmemBytes = 1024 + 8 * kAtom /*Q*/ + 2 * kVTile /*V*/ + 2 * kAtom /*P*/ +
-                              sizeof(Smem);
+constexpr size_t kSmemBytes = 1024 + kRing * kVTile /*V*/ + kRing * kAtom /*P*/ + sizeof(Smem);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+// In-cluster merge, inside the (idle) V region of every split: each split
+// stages its partial output of every head, normalised by its own row sum and
+// rounded to fp16, grouped by the split that merges the head ([owner r][head hh
+// of r's share][512], 1 KB rows whose 16-byte chunks are swizzled by hh), with
+// its (max, sum) pairs; bulk copies then move each group into its owner's
+// receive area ([source split r][hh][512]); the owner merges its heads.
+constexpr uint32_t kMergeSendOff = 0;               // bytes into the V region
+constexpr uint32_t kMergeSendMlOff = 72 * 1024;
+constexpr uint32_t kMergeRecvOff = 76 * 1024;
+constexpr uint32_t kMergeRecvMlOff = 148 * 1024;
+constexpr uint32_t kMergeWtsOff = 152 * 1024;
+static_assert(kMergeWtsOff + 32 * kMaxClusterSplits * sizeof(float) <= (size_t)kRing * kVTile,
+              "merge staging fits in the V region");
+// heads each split of a cluster of ns merges, and the 16-byte-padded bytes of
+// their (max, sum) pairs
+__host__ __device__ constexpr int merge_share(int ns) { return (kHB + ns - 1) / ns; }
+__host__ __device__ constexpr uint32_t merge_ml_bytes(int ns) {
+  return (uint32_t)((merge_share(ns) * 8 + 15) / 16 * 16);
+}
+static_assert(3 * merge_share(3) * 1024 <= 72 * 1024 && 8 * merge_share(8) * 1024 <= 72 * 1024 &&
+                  5 * merge_share(5) * 1024 <= 72 * 1024 && 7 * merge_share(7) * 1024 <= 72 * 1024,
+              "a send or receive area holds every split's share");
+static_assert(kMaxClusterSplits * 176 <= 4 * 1024, "(max, sum) areas");
 
 // byte offset of 16-byte chunk c (0..7) of row r in a [rows][128 B] swizzled block
 __device__ __forceinline__ int swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
@@ -93,11 +127,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// One MMA with each descriptor given as its low word (start address and
-// leading offset: advancing it by (bytes >> 4) cannot carry out, shared-memory
-// addresses being below 2^18) and a common high word.
-__device__ __forceinline__ void mma_f16_lo(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi_a,
-                                           uint32_t hi_b, uint32_t idesc, uint32_t acc) {
+// One MMA, both operands in shared memory, each descriptor given as its low
+// word (start address and leading offset: advancing it by (bytes >> 4) cannot
+// carry out, shared-memory addresses being below 2^18) and a common high word.
+__device__ __forceinline__ void mma_ss(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi_a,
+                                       uint32_t hi_b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
       "setp.ne.b32 p, %6, 0;\n\t"
@@ -106,6 +140,34 @@ __device__ __forceinline__ void mma_f16_lo(uint32_t d, uint32_t a_lo, uint32_t b
       "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d),
       "r"(a_lo), "r"(b_lo), "r"(hi_a), "r"(hi_b), "r"(idesc), "r"(acc)
       : "memory");
+}
+
+// One MMA with A in tensor memory (the same lanes as the accumulator) and B in
+// shared memory.
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi_b,
+                                       uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(b_lo), "r"(hi_b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 16-byte shared-memory accesses by 32-bit shared address
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -123,6 +185,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
 }
 
 // 8 E2M1 codes (one 32-bit word, low nibble first) times their 8 E4M3 scales
@@ -166,27 +233,29 @@ struct AttnParams {
   int cluster_merge;   // the splits of a (row, head block) form a cluster and merge in DSMEM
 };
 
-// float4 chunk c (0..127) of head row h of the fp32 partial staged in the
-// V region; the chunk index is swizzled with the row so that the 16 rows
-// written at once by a warp fall on different banks
-__device__ __forceinline__ int stage_off(int h, int c) { return h * kD + ((c ^ (h & 7)) << 2); }
-
-// 64 columns c0 .. c0 + 63 of head row h of a split's partial O, times f, into
-// the fp32 staging area (the idle V region) that the cluster merge reads
-__device__ __forceinline__ void stage_partial64(float* stage, int h, int c0, const float (&o)[64],
-                                                float f) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c)
-    *reinterpret_cast<float4*>(stage + stage_off(h, c0 / 4 + c)) =
-        make_float4(f * o[4 * c], f * o[4 * c + 1], f * o[4 * c + 2], f * o[4 * c + 3]);
-}
-
 // Raw bytes a producer lane holds for one entry: the codes (8 B) and scales
 // (16 B) of dims 16u .. 16u+15 and of dims 256+16u .. 256+16u+15.
 struct Raw {
   uint2 c[2];
   uint4 s[2];
 };
+
+// The columns of the O accumulator a warp writes out at the end: its quadrant's
+// softmax warp takes chunks 0-2 of 32 columns, producer warp q (q < 4) chunks
+// 3-5 and producer warp q + 4 chunks 6-7 (a 16x32bx2 load covers chunk c and
+// chunk c + 8, 256 columns apart).
+__device__ __forceinline__ void out_chunks(int warp, int& c_begin, int& c_end) {
+  if (warp > kMmaWarp) {
+    c_begin = 0;
+    c_end = 3;
+  } else if (warp < 4) {
+    c_begin = 3;
+    c_end = 6;
+  } else {
+    c_begin = 6;
+    c_end = 8;
+  }
+}
 
 // kG16: the cache is in the pages' own layout, one E4M3 scale per 16 channels
 // stored after the entry's codes (288 bytes per entry), instead of one scale
@@ -196,10 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* qs = base;                              // [8 atoms][64 heads][128 B]
-  uint8_t* vs = qs + 8 * kAtom;                    // [2 buffers][8 atoms][64 entries][128 B]
-  uint8_t* ps = vs + 2 * kVTile;                   // [2 buffers][64 heads][128 B]
-  Smem& sm = *reinterpret_cast<Smem*>(ps + 2 * kAtom);
+  uint8_t* vs = base;                              // [3 buffers][8 atoms][64 entries][128 B]
+  uint8_t* ps = vs + kRing * kVTile;               // [3 buffers][64 heads][128 B]
+  Smem& sm = *reinterpret_cast<Smem*>(ps + kRing * kAtom);
   volatile int* abort_flag = &sm.abort_flag;
 
   const size_t row = blockIdx.x;
@@ -213,30 +281,38 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.bar.q_full, 4);
+    mbar_init(&sm.bar.q_ld, 1);
+    mbar_init(&sm.bar.q_conv, kProducerWarps);
+    mbar_init(&sm.bar.q_full, kProducerWarps);
+    mbar_init(&sm.bar.q_free, kProducerWarps);
     mbar_init(&sm.bar.o_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(&sm.bar.recv, 1);
+    for (int i = 0; i < kRing; ++i) {
       mbar_init(&sm.bar.v_full[i], kProducerWarps);
       mbar_init(&sm.bar.v_free[i], 1);
       mbar_init(&sm.bar.s_full[i], 1);
       mbar_init(&sm.bar.p_full[i], 4);
-      mbar_init(&sm.bar.p_free[i], 1);
     }
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_slot, kTmemCols);
-  // the block's 64 query rows (64 KB) into L2 now: the softmax warps read them
-  // in two dependent batches while the producers wait for their first rows
-  for (int i = threadIdx.x; i < nh * (kD * 2 / 128); i += kThreads) {
-    const uint16_t* qr = p.q + ((row * p.Hq) + h0 + i / 8) * kD + (i % 8) * 64;
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(qr));
-  }
   pdl_wait_and_release();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) {
+    // the block's query rows (1 KB each, contiguous) into V slot 2 in one bulk copy
+    const uint32_t qbytes = (uint32_t)nh * kD * 2;
+    mbar_arrive_expect_tx(&sm.bar.q_ld, qbytes);
+    bulk_load(vs + 2 * kVTile, p.q + ((row * p.Hq) + h0) * kD, qbytes, &sm.bar.q_ld);
+  }
   const uint32_t tmem = sm.tmem_slot;
+  const uint32_t vs_s = smem_u32(vs), ps_s = smem_u32(ps);
+  const int quad = warp & 3;
+  const uint32_t lanes_s = (uint32_t)(quad * 32) << 16;        // S and Q rows: lanes 0-15
+  const uint32_t lanes_o = (uint32_t)(quad * 32 + 16) << 16;   // O rows: lanes 16-31
+  float m_ref = -INFINITY, l = 0.0f;    // softmax threads: the head's maximum, partial row sum
 
   if (warp < kProducerWarps) {
     // ------------------------------------------------------------ gather + dequantise
@@ -286,36 +362,142 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         }
       }
     };
-    auto load_raw = [&](int ids, Raw (&r)[4]) {
+    // half hf of a warp's share of a tile: rounds 2 hf and 2 hf + 1 (four entries)
+    auto load_half = [&](int ids, Raw (&r)[2], int hf) {
 #pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int id = __shfl_sync(0xffffffffu, ids, 2 * rr + half);
+      for (int k = 0; k < 2; ++k) {
+        const int id = __shfl_sync(0xffffffffu, ids, 2 * (2 * hf + k) + half);
         if (id >= 0) {
           const uint8_t* pr = pk_b + (size_t)id * kRowBytes + 8 * u;
-          r[rr].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
-          r[rr].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
+          r[k].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
+          r[k].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
           if (kG16) {
             // dims 16u .. 16u+15 are group u, dims 256+16u .. group 16+u: one
             // scale byte each, repeated for the eight dims of a dequantised chunk
             const uint8_t* sr = pk_b + (size_t)id * kRowBytes + kD / 2 + u;
             const uint32_t s0 = 0x01010101u * __ldg(sr), s1 = 0x01010101u * __ldg(sr + 16);
-            r[rr].s[0] = make_uint4(s0, s0, s0, s0);
-            r[rr].s[1] = make_uint4(s1, s1, s1, s1);
+            r[k].s[0] = make_uint4(s0, s0, s0, s0);
+            r[k].s[1] = make_uint4(s1, s1, s1, s1);
           } else {
             const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + 16 * u;
-            r[rr].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
-            r[rr].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
+            r[k].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
+            r[k].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
           }
         } else {
-          r[rr].c[0] = r[rr].c[1] = make_uint2(0, 0);
-          r[rr].s[0] = r[rr].s[1] = make_uint4(0, 0, 0, 0);
+          r[k].c[0] = r[k].c[1] = make_uint2(0, 0);
+          r[k].s[0] = r[k].s[1] = make_uint4(0, 0, 0, 0);
         }
+      }
+    };
+    auto dequant_half = [&](const Raw (&r)[2], uint4 (&d)[2][4]) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          d[k][2 * hh] = dq8(r[k].c[hh].x, r[k].s[hh].x, r[k].s[hh].y);
+          d[k][2 * hh + 1] = dq8(r[k].c[hh].y, r[k].s[hh].z, r[k].s[hh].w);
+        }
+    };
+    auto store_half = [&](uint32_t tile, const uint4 (&d)[2][4], int hf) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = warp * 8 + 2 * (2 * hf + k) + half;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          // dims 256 hh + 16 u .. + 15: atom 4 hh + u / 4, chunks 2 (u % 4) and 2 (u % 4) + 1;
+          // the two rows of a store differ in parity, so its 32 lanes cover
+          // all eight 16-byte bank groups four times
+          const uint32_t dst = tile + (uint32_t)((4 * hh + (u >> 2)) * kAtom);
+          const int c = (u & 3) * 2;
+          sts128(dst + swz(e, c), d[k][2 * hh]);
+          sts128(dst + swz(e, c + 1), d[k][2 * hh + 1]);
+        }
+      }
+    };
+    // ---- Q into tensor memory (lanes 0-15, columns 192 + d/2). The block's
+    // query rows arrive by one bulk copy into V slot 2. Producer warps w and
+    // w + 4 convert quadrant w % 4's 16 rows in place, 8 rows each, a row at a
+    // time with all 32 lanes: bf16 -> fp16 scaled per head by a power of two (so
+    // every bf16 bit survives), 16-byte chunk c of row hh stored at chunk
+    // c ^ (hh & 7). Then thread (h, ch) of warp w moves dims 256 ch + 128 (w / 4)
+    // .. + 127 of row h into tensor memory. This overlaps the first gathers.
+    auto stage_q = [&]() {
+      const uint32_t qsm = vs_s + 2 * kVTile;
+      bool ok = mbar_wait_warp(&sm.bar.q_ld, 0, abort_flag);
+      if (ok) {
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+          const int hh = quad * 16 + (warp >> 2) * 8 + i;
+          if (hh >= nh) break;                                 // warp-uniform
+          const uint32_t qr = qsm + hh * 1024;
+          const uint4 a = lds128(qr + 16 * lane);
+          const uint4 c = lds128(qr + 512 + 16 * lane);
+          const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+          float amax = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
+                                     fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          // amax < 2^ex with ex from the exponent field; scaling by 2^e, e = 15 - ex,
+          // keeps every magnitude below 2^15 and is exact (clamped to |e| <= 100)
+          int ex2 = 0;
+          if (amax > 0.0f && isfinite(amax)) {
+            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+            ex2 = min(100, max(-100, 15 - ex));
+          }
+          const float up = __uint_as_float((uint32_t)(127 + ex2) << 23);
+          uint32_t f[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            f[k] = pack_half2(__uint_as_float(w[k] << 16) * up,
+                              __uint_as_float(w[k] & 0xffff0000u) * up);
+          __syncwarp();                                        // the row is read before it is rewritten
+          sts128(qr + ((lane ^ (hh & 7)) << 4), make_uint4(f[0], f[1], f[2], f[3]));
+          sts128(qr + (((32 + lane) ^ (hh & 7)) << 4), make_uint4(f[4], f[5], f[6], f[7]));
+          if (lane == 0) sm.qdown[hh] = __uint_as_float((uint32_t)(127 - ex2) << 23);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.bar.q_conv);
+      ok = mbar_wait_warp(&sm.bar.q_conv, 0, abort_flag) && ok;
+      const int h = quad * 16 + (lane & 15), ch = lane >> 4;
+#pragma unroll 1
+      for (int i = 2 * (warp >> 2); i < 2 * (warp >> 2) + 2; ++i) {
+        uint32_t pk[32];
+        if (ok && h < nh) {
+          const uint32_t qr = qsm + h * 1024;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int cl = 32 * ch + 8 * i + j;                // logical 16-byte chunk of the row
+            const uint4 v = lds128(qr + ((cl ^ (h & 7)) << 4));
+            pk[4 * j] = v.x;
+            pk[4 * j + 1] = v.y;
+            pk[4 * j + 2] = v.z;
+            pk[4 * j + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = 0u;
+        }
+        // threads 0-15: columns 192 + 32 i + j (dims 64 i + 2 j, + 1); threads
+        // 16-31: 128 columns further (dims 256 + ...)
+        tmem_st16x2_32<128>(tmem + lanes_s + kTmemQ + 32u * i, pk);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sm.bar.q_full);
+        mbar_arrive(&sm.bar.q_free);
       }
     };
 
     // Indices loaded three tiles ahead (and checked a tile later, when the load
-    // has landed), rows prefetched into L2 two tiles ahead, raw bytes loaded one
-    // tile ahead: nothing on a producer's path waits for a load it just issued.
+    // has landed), rows prefetched into L2 two tiles ahead, and the next tile's
+    // raw bytes loaded while this tile is dequantised (half by half), so a
+    // producer never waits for a load it has just issued.
     int id_cur = check_index(fetch_index(0));
     int id_next = check_index(fetch_index(1));
     int id_after = check_index(fetch_index(2));
@@ -323,35 +505,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     prefetch_rows(id_cur);
     prefetch_rows(id_next);
     prefetch_rows(id_after);
-    Raw raw[4];
-    load_raw(id_cur, raw);
-    bool go = true;
-    for (int t = 0; go && t < nt; ++t) {
-      const int buf = t & 1;
-      // the buffer (and its valid bits) is free once P(t-2) V(t-2) has completed
-      if (!mbar_wait_warp(&sm.bar.v_free[buf], ((t >> 1) & 1) ^ 1, abort_flag)) {
-        go = false;
-        break;
-      }
+    Raw ra[2], rb[2];
+    load_half(id_cur, ra, 0);
+    load_half(id_cur, rb, 1);
+    stage_q();
+    for (int t = 0; t < nt; ++t) {
+      const int buf = t % kRing;
+      uint4 dq[2][4];
+      dequant_half(ra, dq);
+      load_half(id_next, ra, 0);
       const uint32_t vb = __ballot_sync(0xffffffffu, id_cur >= 0);   // lanes 8-31 hold -1
+      // the slot (and its valid bits) is free once P(t-3) V(t-3) has completed;
+      // slot 2 first holds the query block until the softmax warps have read it
+      if (!mbar_wait_warp(&sm.bar.v_free[buf], ((t / kRing) & 1) ^ 1, abort_flag)) break;
+      if (t == 2 && !mbar_wait_warp(&sm.bar.q_free, 0, abort_flag)) break;
       if (lane == 0) reinterpret_cast<uint8_t*>(sm.valid[buf])[warp] = (uint8_t)vb;
-      uint8_t* tile = vs + buf * kVTile;
-#pragma unroll
-      for (int rr = 0; rr < 4; ++rr) {
-        const int e = warp * 8 + 2 * rr + half;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          // dims 256 hh + 16 u .. + 15: atom 4 hh + u / 4, chunks 2 (u % 4) and 2 (u % 4) + 1;
-          // the two rows of a store differ in parity, so its 32 lanes cover
-          // all eight 16-byte bank groups four times
-          uint8_t* dst = tile + (4 * hh + (u >> 2)) * kAtom;
-          const int c = (u & 3) * 2;
-          const uint2 cw = raw[rr].c[hh];
-          const uint4 sw = raw[rr].s[hh];
-          *reinterpret_cast<uint4*>(dst + swz(e, c)) = dq8(cw.x, sw.x, sw.y);
-          *reinterpret_cast<uint4*>(dst + swz(e, c + 1)) = dq8(cw.y, sw.z, sw.w);
-        }
-      }
+      const uint32_t tile = vs_s + (uint32_t)(buf * kVTile);
+      store_half(tile, dq, 0);
+      dequant_half(rb, dq);
+      load_half(id_next, rb, 1);
+      store_half(tile, dq, 1);
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.v_full[buf]);
@@ -361,59 +534,37 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       id_cur = id_next;
       id_next = id_after;
       id_after = id_far_checked;
-      load_raw(id_cur, raw);
-    }
-    if (p.cluster_merge && go) {
-      // Staging of the split's partial for the merge, shared with the softmax
-      // warps: producer warps q and q + 4 take columns 192 (w >> 2) .. + 191 of
-      // the 16 O rows of TMEM quadrant q (heads 16 q ..), the softmax warp of
-      // the quadrant the last 128. x 2^8 undoes the factor the dequantised
-      // values carry; an empty split is skipped by the merge, whatever it stages.
-      if (mbar_wait_warp(&sm.bar.o_full, 0, abort_flag)) {
-        tc_fence_after();
-        const int quad = warp & 3;
-        const int hq = quad * 16 + (lane & 15);
-        const uint32_t la = (uint32_t)(quad * 32) << 16;
-#pragma unroll 1
-        for (int k = 0; k < 3; ++k) {
-          const int c0 = (warp >> 2) * 192 + k * 64;
-          float o[64];
-          tmem_ld_64(tmem + la + c0, o);
-          if (lane < 16 && hq < nh) stage_partial64(reinterpret_cast<float*>(vs), hq, c0, o, 256.0f);
-        }
-      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_f16(64, kT, 0);
       const uint32_t id_o = idesc_f16(64, 256, 1);
-      const uint64_t qd = desc_sw128(smem_u32(qs), 16, 1024);
       const uint64_t vk = desc_sw128(smem_u32(vs), 16, 1024);       // V tile as K-major B
       const uint64_t vn = desc_sw128(smem_u32(vs), kAtom, 1024);    // V tile as N-major B
       const uint64_t pd = desc_sw128(smem_u32(ps), 16, 1024);       // P as K-major A
       bool ok = mbar_wait(&sm.bar.q_full, 0, abort_flag);
-      // S(t) into buffer t & 1: lanes 16-31, columns 64 (t & 1) .. + 63
+      tc_fence_after();
+      // S(t) into buffer t % 3: lanes 0-15, columns 64 (t % 3) .. + 63
       auto issue_s = [&](int t) -> bool {
-        const int buf = t & 1;
-        if (!mbar_wait(&sm.bar.v_full[buf], (t >> 1) & 1, abort_flag)) return false;
+        const int buf = t % kRing;
+        if (!mbar_wait(&sm.bar.v_full[buf], (t / kRing) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t d = tmem + (16u << 16) + 64u * buf;
-        const uint32_t q_lo = (uint32_t)qd, q_hi = (uint32_t)(qd >> 32);
+        const uint32_t d = tmem + 64u * buf;
         const uint32_t v_lo = (uint32_t)vk + (uint32_t)((buf * kVTile) >> 4);
         const uint32_t v_hi = (uint32_t)(vk >> 32);
 #pragma unroll
         for (int a = 0; a < 8; ++a)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16_lo(d, q_lo + (uint32_t)((a * kAtom + kk * 32) >> 4),
-                       v_lo + (uint32_t)((a * kAtom + kk * 32) >> 4), q_hi, v_hi, id_s,
-                       (a > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(d, tmem + kTmemQ + 8u * (4 * a + kk),
+                   v_lo + (uint32_t)((a * kAtom + kk * 32) >> 4), v_hi, id_s,
+                   (a > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar.s_full[buf]);
         return true;
       };
       auto issue_pv = [&](int t) {
-        const int buf = t & 1;
+        const int buf = t % kRing;
         tc_fence_after();
         const uint32_t p_lo = (uint32_t)pd + (uint32_t)((buf * kAtom) >> 4);
         const uint32_t p_hi = (uint32_t)(pd >> 32);
@@ -424,28 +575,29 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int ks = 0; ks < kT / 16; ++ks)
-            mma_f16_lo(tmem + 256u * h, p_lo + (uint32_t)((ks * 32) >> 4),
-                       n_lo + (uint32_t)((h * 4 * kAtom + ks * 2048) >> 4), p_hi, n_hi, id_o,
-                       ks > 0 ? 1u : acc0);
+            mma_ss(tmem + (16u << 16) + 256u * h, p_lo + (uint32_t)((ks * 32) >> 4),
+                   n_lo + (uint32_t)((h * 4 * kAtom + ks * 2048) >> 4), p_hi, n_hi, id_o,
+                   ks > 0 ? 1u : acc0);
+        // the V slot, and (through the in-order completion of later MMAs) the P
+        // buffer, are free once this has completed
         mma_commit(&sm.bar.v_free[buf]);
-        mma_commit(&sm.bar.p_free[buf]);
       };
-      if (ok && nt > 0) ok = issue_s(0);
-      if (ok && nt > 1) ok = issue_s(1);
+      for (int t = 0; ok && t < min(nt, kRing - 1); ++t) ok = issue_s(t);
       // Then whichever is ready first: P(t) V(t) once the softmax published P(t),
-      // or S(t') (t' <= t + 1: its S and P buffers were released by P(t'-2) V(t'-2))
-      // once the producers published its tile. Polling is bounded like mbar_wait.
-      int next_pv = 0, next_s = 2;
+      // or S(t') (t' <= t + 2: its S and P buffers were released by the issue of
+      // P(t'-3) V(t'-3), which completes before S(t')) once the producers
+      // published its tile. Polling is bounded like mbar_wait.
+      int next_pv = 0, next_s = min(nt, kRing - 1);
       const uint64_t t0 = global_ns();
       uint32_t spins = 0;
       while (ok && next_pv < nt) {
         bool did = false;
-        if (mbar_test_wait(&sm.bar.p_full[next_pv & 1], (next_pv >> 1) & 1)) {
+        if (mbar_test_wait(&sm.bar.p_full[next_pv % kRing], (next_pv / kRing) & 1)) {
           issue_pv(next_pv++);
           did = true;
         }
-        if (next_s < nt && next_s <= next_pv + 1 &&
-            mbar_test_wait(&sm.bar.v_full[next_s & 1], (next_s >> 1) & 1)) {
+        if (next_s < nt && next_s <= next_pv + kRing - 1 &&
+            mbar_test_wait(&sm.bar.v_full[next_s % kRing], (next_s / kRing) & 1)) {
           ok = issue_s(next_s++);
           did = true;
         }
@@ -458,81 +610,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         }
       }
       mma_commit(&sm.bar.o_full);
-      // nothing may be in flight when TMEM is released
+      // nothing may be in flight when tensor memory is released
       mbar_wait(&sm.bar.o_full, 0, abort_flag);
     }
   } else {
-    // ------------------------------------------------------------ Q, softmax, epilogue
-    const int quad = warp & 3;
-    const int sw = warp - (kMmaWarp + 1);            // 0..3: Q heads 16 sw .. 16 sw + 15
-    const bool s_owner = lane >= 16;                 // S rows live in lanes 16-31
-    const int h = quad * 16 + (lane & 15);           // head of this lane's S (or O) row
-    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    // ---- Q, scaled per head by a power of two so that its bf16 values keep
-    // every bit in fp16; two batches of eight heads per warp
-#pragma unroll 1
-    for (int bt = 0; bt < 2; ++bt) {
-      uint4 qraw[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int hh = sw * 16 + bt * 8 + j;
-        if (hh < nh) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(p.q + ((row * p.Hq) + h0 + hh) * kD + lane * 16);
-          qraw[2 * j] = __ldg(src);
-          qraw[2 * j + 1] = __ldg(src + 1);
-        } else {
-          qraw[2 * j] = make_uint4(0, 0, 0, 0);
-          qraw[2 * j + 1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int hh = sw * 16 + bt * 8 + j;
-        const uint32_t w[8] = {qraw[2 * j].x, qraw[2 * j].y, qraw[2 * j].z, qraw[2 * j].w,
-                               qraw[2 * j + 1].x, qraw[2 * j + 1].y, qraw[2 * j + 1].z,
-                               qraw[2 * j + 1].w};
-        float vals[16];
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          vals[2 * i] = __uint_as_float(w[i] << 16);
-          vals[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-          amax = fmaxf(amax, fmaxf(fabsf(vals[2 * i]), fabsf(vals[2 * i + 1])));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        // amax < 2^ex with ex from the exponent field; scaling by 2^e, e = 15 - ex,
-        // keeps every magnitude below 2^15 and is exact (clamped to |e| <= 100)
-        int ex2 = 0;
-        if (amax > 0.0f && isfinite(amax)) {
-          const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-          ex2 = min(100, max(-100, 15 - ex));
-        }
-        const float up = __uint_as_float((uint32_t)(127 + ex2) << 23);
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) pk[i] = pack_half2(vals[2 * i] * up, vals[2 * i + 1] * up);
-        const int atom = lane >> 2, c0 = (lane & 3) * 2;
-        uint8_t* dst = qs + atom * kAtom;
-        *reinterpret_cast<uint4*>(dst + swz(hh, c0)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(dst + swz(hh, c0 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        const float down = __uint_as_float((uint32_t)(127 - ex2) << 23);
-        // x 2^8: the dequantised keys/values carry a factor 2^-8
-        if (lane == 0) sm.head_scale[hh] = hh < nh ? p.softmax_scale * kLog2e * down * 256.0f : 0.0f;
-      }
-    }
-    fence_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.bar.q_full);
-    // every softmax warp reads the scales of its own heads after all four staged Q
+    // ------------------------------------------------------------ Q, softmax
+    const int hl = lane & 15, ch = lane >> 4;        // head in the quadrant, half of the tile
+    const int h = quad * 16 + hl;                    // head of this thread within the block
+    // the producers stage Q (and the per-head scales) first
     bool ok = mbar_wait_warp(&sm.bar.q_full, 0, abort_flag);
-    const float hs = sm.head_scale[h];
-    float m_ref = -INFINITY, l = 0.0f;    // meaningful in the S lanes
+    // x 2^8: the dequantised keys/values carry a factor 2^-8
+    const float hs = (ok && h < nh) ? p.softmax_scale * kLog2e * sm.qdown[h] * 256.0f : 0.0f;
     for (int t = 0; ok && t < nt; ++t) {
-      const int buf = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      // S(t) complete also means P(t-2) V(t-2) is: P buffer t & 1 is free; the
+      const int buf = t % kRing;
+      const uint32_t ph = (t / kRing) & 1;
+      // S(t) complete also means P(t-3) V(t-3) is: P buffer t % 3 is free; the
       // valid bits of tile t were written before its V tile was published
       ok = mbar_wait_warp(&sm.bar.v_full[buf], ph, abort_flag) &&
            mbar_wait_warp(&sm.bar.s_full[buf], ph, abort_flag);
@@ -540,245 +632,294 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       tc_fence_after();
       const uint32_t vw0 = sm.valid[buf][0], vw1 = sm.valid[buf][1];
       const bool all_valid = (vw0 & vw1) == 0xffffffffu;     // the same for every lane
-      float y[64];
-      tmem_ld_64(tmem + lane_addr + 64u * buf, y);
-      // logits in the log2 domain relative to the current reference maximum,
-      // and their maximum over the selected entries
+      const uint32_t vw = ch ? vw1 : vw0;                      // entries 32 ch .. 32 ch + 31
+      float y[32];
+      tmem_ld16x2_32<32>(tmem + lanes_s + 64u * buf, y);
+      // logits in the log2 domain and their maximum over the selected entries
       float xmax = -INFINITY;
       if (all_valid) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          y[j] = fmaf(y[j], hs, -m_ref);
+        for (int j = 0; j < 32; ++j) {
+          y[j] *= hs;
           xmax = fmaxf(xmax, y[j]);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          y[j] = fmaf(y[j], hs, -m_ref);
-          const bool v = (((j < 32 ? vw0 : vw1) >> (j & 31)) & 1u) != 0u;
-          xmax = fmaxf(xmax, v ? y[j] : -INFINITY);
+        for (int j = 0; j < 32; ++j) {
+          y[j] *= hs;
+          xmax = fmaxf(xmax, ((vw >> j) & 1u) ? y[j] : -INFINITY);
         }
       }
+      xmax = fmaxf(xmax, __shfl_xor_sync(0xffffffffu, xmax, 16));
       // lazy reference maximum: raise it only when P would exceed 2^8 (always on
       // the first tile with a selected entry, where the reference is -inf)
-      const bool raise = s_owner && xmax > kRescaleSlack;
-      float alpha = 1.0f;
-      const float m_old = m_ref;
+      const bool raise = xmax > m_ref + kRescaleSlack;
       if (__any_sync(0xffffffffu, raise)) {
-        tmem_ld_64(tmem + lane_addr + 64u * buf, y);
-        float ymax = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          y[j] *= hs;
-          const bool v = (((j < 32 ? vw0 : vw1) >> (j & 31)) & 1u) != 0u;
-          ymax = fmaxf(ymax, v ? y[j] : -INFINITY);
-        }
+        float alpha = 1.0f;
+        const bool had = m_ref != -INFINITY;
         if (raise) {
-          alpha = m_ref == -INFINITY ? 0.0f : exp2f(m_ref - ymax);
-          m_ref = ymax;
+          alpha = had ? fast_exp2(m_ref - xmax) : 0.0f;
+          m_ref = xmax;
           l *= alpha;
         }
-#pragma unroll
-        for (int j = 0; j < 64; ++j) y[j] -= m_ref;
-      }
-      // O (lanes 0-15) is rescaled by its S lane's factor once P(t-1) V(t-1) is done
-      const bool need = s_owner && alpha != 1.0f && m_old != -INFINITY;
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
-        // the TMEM loads and stores below cover all 32 lanes of the quadrant:
-        // wait until nothing writes them, i.e. P(t-1) V(t-1) (O, lanes 0-15) and
-        // S(t+1) (the other S buffer, lanes 16-31, stored back unchanged) are done
-        ok = mbar_wait_warp(&sm.bar.p_free[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag);
-        if (ok && t + 1 < nt)
-          ok = mbar_wait_warp(&sm.bar.s_full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const float a_o = __shfl_down_sync(0xffffffffu, need ? alpha : 1.0f, 16);
-        const float f = s_owner ? 1.0f : a_o;
+        // O (lanes 16-31) holds P(0..t-1) V: rescale it by the head's factor once
+        // P(t-1) V(t-1) has completed (P(t) V(t) waits for this tile's P)
+        const bool need = raise && had;
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
+          ok = mbar_wait_warp(&sm.bar.v_free[(t - 1) % kRing], ((t - 1) / kRing) & 1,
+                              abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const float f = need ? alpha : 1.0f;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-          float o[32];
-          tmem_ld_32(tmem + lane_addr + c0, o);
+          for (int c0 = 0; c0 < kD / 2; c0 += 32) {
+            float o[32];
+            tmem_ld16x2_32<256>(tmem + lanes_o + c0, o);
+            uint32_t ow[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= f;
-          tmem_st_32(tmem + lane_addr + c0, o);
+            for (int c = 0; c < 32; ++c) ow[c] = __float_as_uint(o[c] * f);
+            tmem_st16x2_32<256>(tmem + lanes_o + c0, ow);
+          }
         }
       }
-      // P = 2^y in fp16 (y <= 8) as the A operand of P V, and the row sum
-      const bool live = s_owner && m_ref != -INFINITY;
-      uint8_t* prow = ps + buf * kAtom;
+      // P = 2^(y - m) in fp16 (<= 2^8) as the A operand of P V, and the row sum
+      const bool live = m_ref != -INFINITY;
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = 8 * c + 2 * u;
-          const uint32_t vw = j < 32 ? vw0 : vw1;
-          const bool v0 = live && (all_valid || ((vw >> (j & 31)) & 1u));
-          const bool v1 = live && (all_valid || ((vw >> ((j + 1) & 31)) & 1u));
-          const float p0 = v0 ? fast_exp2(y[j]) : 0.0f;
-          const float p1 = v1 ? fast_exp2(y[j + 1]) : 0.0f;
-          l += p0 + p1;
-          pk[u] = pack_half2(p0, p1);
-        }
-        if (s_owner)
-          *reinterpret_cast<uint4*>(prow + swz(h, c)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int j = 0; j < 32; j += 2) {
+        const bool v0 = live && (all_valid || ((vw >> j) & 1u));
+        const bool v1 = live && (all_valid || ((vw >> (j + 1)) & 1u));
+        const float p0 = v0 ? fast_exp2(y[j] - m_ref) : 0.0f;
+        const float p1 = v1 ? fast_exp2(y[j + 1] - m_ref) : 0.0f;
+        l += p0 + p1;
+        pk[j / 2] = pack_half2(p0, p1);
       }
+      const uint32_t prow = ps_s + (uint32_t)(buf * kAtom);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        sts128(prow + swz(h, 4 * ch + c),
+               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.p_full[buf]);
     }
-    // epilogue: O rows live in lanes 0-15; fetch m and l from the S lane (+16)
-    const float m_o = __shfl_down_sync(0xffffffffu, m_ref, 16);
-    const float l_o = __shfl_down_sync(0xffffffffu, l, 16);
-    ok = mbar_wait_warp(&sm.bar.o_full, 0, abort_flag) && ok;
-    if (ok) {
-      tc_fence_after();
-      const bool o_owner = lane < 16 && h < nh;
-      const size_t slot = (row * p.nhb + hb) * p.nsplit + split;
-      // x 2^8 undoes the 2^-8 carried by the dequantised values; a split with
-      // nothing selected writes zeros whatever the accumulator holds
-      const float f = l_o > 0.0f ? (p.nsplit == 1 ? 256.0f / l_o : 256.0f) : 0.0f;
-#pragma unroll 1
-      for (int c0 = p.cluster_merge ? 384 : 0; c0 < kD; c0 += 64) {
-        float o[64];
-        tmem_ld_64(tmem + lane_addr + c0, o);
-        if (!o_owner) continue;
-        if (p.nsplit == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + h) * kD + c0);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              __nv_bfloat162 bb = __floats2bfloat162_rn(l_o > 0.0f ? o[8 * c + 2 * u] * f : 0.0f,
-                                                        l_o > 0.0f ? o[8 * c + 2 * u + 1] * f : 0.0f);
-              w[u] = *reinterpret_cast<uint32_t*>(&bb);
-            }
-            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else if (p.cluster_merge) {
-          // partial into the idle V region; merged over DSMEM below
-          stage_partial64(reinterpret_cast<float*>(vs), h, c0, o, 256.0f);
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + c0);
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            dst[c] = l_o > 0.0f ? make_float4(f * o[4 * c], f * o[4 * c + 1], f * o[4 * c + 2],
-                                              f * o[4 * c + 3])
-                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        }
-      }
-      if (lane < 16 && h < nh) {
-        const float2 ml = make_float2(l_o > 0.0f ? m_o : -INFINITY, l_o);
-        if (p.nsplit == 1) {
-          if (p.lse) p.lse[row * p.Hq + h0 + h] = l_o > 0.0f ? (m_o + log2f(l_o)) * kLn2 : -INFINITY;
-        } else if (p.cluster_merge) {
-          sm.ml[h] = ml;
-        } else {
-          p.ws_ml[slot * kHB + h] = ml;
-        }
-      }
-    }
+    const float l_tot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+    if (ch == 0) sm.mlf[h] = make_float2(l_tot > 0.0f ? m_ref : -INFINITY, l_tot);
   }
 
+  // ---------------------------------------------------------------- output
+  // Every warp that reaches a quadrant's O lanes waits for the last P V, then
+  // handles its chunks of the quadrant's 16 heads: the final output (one
+  // split), the partial staged for the in-cluster merge, or the partial in the
+  // workspace. x 2^8 undoes the 2^-8 carried by the dequantised values.
+  const bool writer = warp != kMmaWarp;
+  bool have_o = false;
+  if (writer) have_o = mbar_wait_warp(&sm.bar.o_full, 0, abort_flag);
+  tc_fence_before();
+  __syncthreads();                 // O is final, the (max, sum) pairs are in shared memory
+  tc_fence_after();
+  const int ns = p.nsplit;
+  const int share = merge_share(ns);                   // heads each split of a cluster merges
+  const uint32_t mlb = merge_ml_bytes(ns);
+  if (p.cluster_merge && threadIdx.x == 0)
+    mbar_arrive_expect_tx(&sm.bar.recv, (uint32_t)(ns - 1) * ((uint32_t)share * 1024u + mlb));
+  if (writer && have_o) {
+    const int hl = lane & 15, ch = lane >> 4;
+    const int h = quad * 16 + hl;
+    const float2 mlh = sm.mlf[h];
+    const float l_tot = mlh.y;
+    int cb, ce;
+    out_chunks(warp, cb, ce);
+    const size_t slot = (row * p.nhb + hb) * p.nsplit + split;
+    const int owner = h / share, hh = h - owner * share;
+    const uint32_t send_row = vs_s + kMergeSendOff + (uint32_t)(owner * share + hh) * 1024u;
+#pragma unroll 1
+    for (int c = cb; c < ce; ++c) {
+      float o[32];
+      tmem_ld16x2_32<256>(tmem + lanes_o + 32u * c, o);
+      if (h >= nh) continue;
+      const int d0 = 256 * ch + 32 * c;           // this thread's dims d0 .. d0 + 31
+      if (ns == 1) {
+        const float f = l_tot > 0.0f ? 256.0f / l_tot : 0.0f;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + h) * kD + d0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          dst[k] = make_uint4(pack_bf162(o[8 * k] * f, o[8 * k + 1] * f),
+                              pack_bf162(o[8 * k + 2] * f, o[8 * k + 3] * f),
+                              pack_bf162(o[8 * k + 4] * f, o[8 * k + 5] * f),
+                              pack_bf162(o[8 * k + 6] * f, o[8 * k + 7] * f));
+      } else if (p.cluster_merge) {
+        // normalised by this split's row sum (a convex combination of values,
+        // |o| <= 2688, so fp16 holds it); nothing selected gives zeros
+        const float f = l_tot > 0.0f ? 256.0f / l_tot : 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int cl = d0 / 8 + k;                  // logical 16-byte chunk of the row
+          sts128(send_row + ((cl ^ (hh & 7)) << 4),
+                 make_uint4(pack_half2(o[8 * k] * f, o[8 * k + 1] * f),
+                            pack_half2(o[8 * k + 2] * f, o[8 * k + 3] * f),
+                            pack_half2(o[8 * k + 4] * f, o[8 * k + 5] * f),
+                            pack_half2(o[8 * k + 6] * f, o[8 * k + 7] * f)));
+        }
+      } else {
+        // unnormalised, with the split's (max, sum), for the combine kernel;
+        // a split with nothing selected contributes zeros
+        const float f = l_tot > 0.0f ? 256.0f : 0.0f;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + d0);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(f * o[4 * k], f * o[4 * k + 1], f * o[4 * k + 2],
+                               f * o[4 * k + 3]);
+      }
+    }
+    if (warp > kMmaWarp && ch == 0 && h < nh) {
+      if (ns == 1) {
+        if (p.lse)
+          p.lse[row * p.Hq + h0 + h] =
+              l_tot > 0.0f ? (mlh.x + log2f(l_tot)) * kLn2 : -INFINITY;
+      } else if (p.cluster_merge) {
+        reinterpret_cast<float2*>(vs + kMergeSendMlOff + owner * mlb)[hh] = mlh;
+      } else {
+        p.ws_ml[slot * kHB + h] = mlh;
+      }
+    }
+    if (p.cluster_merge) fence_async_smem();      // the staging is read by bulk copies
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) record_error(p.err, CSA2_ERR_TIMEOUT);
 
   if (p.cluster_merge) {
-    // Split s of the cluster merges heads [s share, (s + 1) share) of all splits'
-    // partials, read over DSMEM: out = sum_r w_r O_r with w_r = 2^(m_r - M) / L,
-    // L = sum_r 2^(m_r - M) l_r, M = max_r m_r. The weights of a head are
-    // computed once (into the idle Q region); then every thread loads its
-    // outputs' partials from all splits before combining them.
+    // Every split has staged its partials and left its V region idle. Split s
+    // sends its group for owner r into r's receive area, slot s, and merges the
+    // heads [s share, (s + 1) share) from its own group and the ones it received:
+    // out = sum_r w_r o_r with o_r the partial normalised by its row sum l_r,
+    // w_r = 2^(m_r - M) l_r / L, L = sum_r 2^(m_r - M) l_r, M = max_r m_r.
     cg::cluster_group cl = cg::this_cluster();
-    cl.sync();                                   // every split's partial is staged
-    const int ns = p.nsplit;
-    const int share = (kHB + ns - 1) / ns;
+    cl.sync();
+    if (threadIdx.x == 0) {
+      const uint32_t recv_bar = smem_u32(&sm.bar.recv);
+      for (int r = 0; r < ns; ++r) {
+        if (r == split) continue;
+        bulk_copy_to_peer(
+            cluster_addr(smem_u32(vs + kMergeRecvOff + (size_t)split * share * 1024), (uint32_t)r),
+            vs + kMergeSendOff + (size_t)r * share * 1024, (uint32_t)share * 1024u,
+            cluster_addr(recv_bar, (uint32_t)r));
+        bulk_copy_to_peer(cluster_addr(smem_u32(vs + kMergeRecvMlOff + split * mlb), (uint32_t)r),
+                          vs + kMergeSendMlOff + r * mlb, mlb, cluster_addr(recv_bar, (uint32_t)r));
+      }
+    }
+    const bool got = mbar_wait_warp(&sm.bar.recv, 0, abort_flag);
     const int hA = split * share, hB = min(nh, hA + share);
     const int nhm = max(0, hB - hA);
-    float* wts = reinterpret_cast<float*>(qs);   // [head - hA][8 splits]
-    for (int i = threadIdx.x; i < nhm; i += kThreads) {
-      const int hh = hA + i;
-      float mv[8], lv[8];
-      float M = -INFINITY;
+    auto part_row = [&](int r, int i) -> uint32_t {
+      return r == split ? vs_s + kMergeSendOff + (uint32_t)(split * share + i) * 1024u
+                        : vs_s + kMergeRecvOff + (uint32_t)(r * share + i) * 1024u;
+    };
+    auto part_ml = [&](int r, int i) -> float2 {
+      return r == split ? reinterpret_cast<const float2*>(vs + kMergeSendMlOff + split * mlb)[i]
+                        : reinterpret_cast<const float2*>(vs + kMergeRecvMlOff + r * mlb)[i];
+    };
+    float* wts = reinterpret_cast<float*>(vs + kMergeWtsOff);    // [own head][8 splits]
+    if (got) {
+      for (int i = threadIdx.x; i < nhm; i += kThreads) {
+        float M = -INFINITY;
+        for (int r = 0; r < ns; ++r) M = fmaxf(M, part_ml(r, i).x);
+        float w[kMaxClusterSplits];
+        float L = 0.0f;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        mv[r] = -INFINITY;
-        lv[r] = 0.0f;
-        if (r < ns) {
-          const float2 ml = cl.map_shared_rank(&sm.ml[hh], r)[0];
-          mv[r] = ml.x;
-          lv[r] = ml.y;
-          M = fmaxf(M, ml.x);
+        for (int r = 0; r < kMaxClusterSplits; ++r) {
+          w[r] = 0.0f;
+          if (r < ns) {
+            const float2 ml = part_ml(r, i);
+            w[r] = (ml.x != -INFINITY && ml.y > 0.0f) ? exp2f(ml.x - M) * ml.y : 0.0f;
+            L += w[r];
+          }
         }
-      }
-      float w[8];
-      float L = 0.0f;
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        w[r] = mv[r] != -INFINITY ? exp2f(mv[r] - M) : 0.0f;
-        L += w[r] * lv[r];
+        for (int r = 0; r < kMaxClusterSplits; ++r) wts[i * kMaxClusterSplits + r] = w[r] * inv;
+        if (p.lse) p.lse[row * p.Hq + h0 + hA + i] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
       }
-      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) wts[i * 8 + r] = w[r] * inv;
-      if (p.lse) p.lse[row * p.Hq + h0 + hh] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
     __syncthreads();
-    const int units = nhm * (kD / 4);
-    constexpr int kBatch = 2;                    // outputs per thread whose loads are in flight together
+    const int units = got ? nhm * (kD / 8) : 0;        // 16-byte chunks of 8 fp16
 #pragma unroll 1
-    for (int base = threadIdx.x; base < units; base += kBatch * kThreads) {
-      float4 v[kBatch][8];
-      float wv[kBatch][8];
+    for (int uo = threadIdx.x; uo < units; uo += kThreads) {
+      const int i = uo / (kD / 8), cl = uo % (kD / 8);
+      const int off = (cl ^ (i & 7)) << 4;
+      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int u = base + j * kThreads;
-        const int i = u / (kD / 4), c = u % (kD / 4);
+      for (int r = 0; r < kMaxClusterSplits; ++r) {
+        if (r < ns) {
+          const float wr = wts[i * kMaxClusterSplits + r];
+          if (wr != 0.0f) {
+            const uint4 v = lds128(part_row(r, i) + off);
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          wv[j][r] = (u < units && r < ns) ? wts[i * 8 + r] : 0.0f;
-          v[j][r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (wv[j][r] != 0.0f) {
-            const float* st = cl.map_shared_rank(reinterpret_cast<float*>(vs), r);
-            v[j][r] = *reinterpret_cast<const float4*>(st + stage_off(hA + i, c));
+            for (int k = 0; k < 4; ++k) {
+              const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
+              acc[2 * k] = fmaf(wr, f2.x, acc[2 * k]);
+              acc[2 * k + 1] = fmaf(wr, f2.y, acc[2 * k + 1]);
+            }
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < kBatch; ++j) {
-        const int u = base + j * kThreads;
-        if (u >= units) break;
-        const int i = u / (kD / 4), c = u % (kD / 4);
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          acc.x = fmaf(wv[j][r], v[j][r].x, acc.x);
-          acc.y = fmaf(wv[j][r], v[j][r].y, acc.y);
-          acc.z = fmaf(wv[j][r], v[j][r].z, acc.z);
-          acc.w = fmaf(wv[j][r], v[j][r].w, acc.w);
-        }
-        __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-        *reinterpret_cast<uint2*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 4 * c) = pk;
-      }
+      *reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 8 * cl) =
+          make_uint4(pack_bf162(acc[0], acc[1]), pack_bf162(acc[2], acc[3]),
+                     pack_bf162(acc[4], acc[5]), pack_bf162(acc[6], acc[7]));
     }
-    cl.sync();                                   // no split leaves while others read it
+    // no split leaves while a bulk copy may still read its staging
+    cl.sync();
   }
+  if (threadIdx.x == 0 && *abort_flag) record_error(p.err, CSA2_ERR_TIMEOUT);
 }
+
+template <bool kG16>
+struct KernelSetup {
+  // cudaFuncSetAttribute and the cluster occupancy query, once per device
+  static cudaError_t prepare(bool* clusters_ok) {
+    static int done[64] = {};
+    static int cluster_fit[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {
+      e = cudaFuncSetAttribute(sparse_attn_tc_kernel<kG16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kMaxClusterSplits, 1, kMaxClusterSplits);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = kMaxClusterSplits;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      cluster_fit[dev] = cudaOccupancyMaxActiveClusters(&n, sparse_attn_tc_kernel<kG16>, &cfg) ==
+                                 cudaSuccess &&
+                             n > 0;
+      (void)cudaGetLastError();
+      done[dev] = 1;
+    }
+    *clusters_ok = cluster_fit[dev] != 0;
+    return cudaSuccess;
+  }
+};
 
 }  // namespace
 
 int sparse_attn_tc_tile() { return kT; }
+int sparse_attn_tc_max_cluster() { return kMaxClusterSplits; }
 
 cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
@@ -806,41 +947,27 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
   p.err = err;
   p.cluster_merge = 0;
   // no block-scale array: rows of the 16-channel layout
-  void (*kernel)(AttnParams) =
-      kv_scale == nullptr ? sparse_attn_tc_kernel<true> : sparse_attn_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  const bool g16 = kv_scale == nullptr;
+  void (*kernel)(AttnParams) = g16 ? sparse_attn_tc_kernel<true> : sparse_attn_tc_kernel<false>;
+  bool clusters_ok = false;
+  cudaError_t e = g16 ? KernelSetup<true>::prepare(&clusters_ok)
+                      : KernelSetup<false>::prepare(&clusters_ok);
   if (e != cudaSuccess) return e;
   dim3 grid(rows, nhb, nsplit);
   if (merged != nullptr) *merged = false;
-  if (nsplit > 1 && nsplit <= 8 && merged != nullptr) {
+  if (nsplit > 1 && nsplit <= kMaxClusterSplits && merged != nullptr && clusters_ok) {
     // the splits of each (row, head block) as one cluster: merged in DSMEM
     p.cluster_merge = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = (unsigned)nsplit;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg) == cudaSuccess &&
-        nclusters > 0) {
-      e = launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream,
-                     dim3(1, 1, (unsigned)nsplit), p);
-      if (e == cudaSuccess) {
-        *merged = true;
-        return cudaSuccess;
-      }
+    e = launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream,
+                   dim3(1, 1, (unsigned)nsplit), p);
+    if (e == cudaSuccess) {
+      *merged = true;
+      return cudaSuccess;
     }
     (void)cudaGetLastError();   // fall back to partials in the workspace
     p.cluster_merge = 0;
   }
+  if (nsplit > 1 && ws_o == nullptr) return cudaErrorInvalidValue;
   return launch_pdl(kernel, grid, dim3(kThreads), kSmemBytes, stream, dim3(1), p);
 }
 
