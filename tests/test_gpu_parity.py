@@ -13,7 +13,8 @@ from fp4_kv_cache_step_b200 import build as libbuild
 from fp4_kv_cache_step_b200 import csa2
 from fp4_kv_cache_step_b200 import workloads as wl
 from fp4_kv_cache_step_b200.runner import DeviceWorkload
-from tests.parity_utils import (assert_attn_close, assert_lse_close, bf16_dev, dev, host)
+from tests.parity_utils import (assert_attn_close, assert_lse_close, bf16_dev, dev, host,
+                                row_vmax)
 
 pytestmark = pytest.mark.gpu
 
@@ -201,9 +202,50 @@ def test_sparse_attn_within_tolerance(B, Tq, Hq, N, K, scale):
     idx[0, 0, :] = -1                                   # a row with nothing selected
     want, want_lse = oracle.sparse_attn(q, packed, sc, idx, scale)
     out, lse = csa2.csa2_sparse_attn(bf16_dev(q), dev(packed), dev(sc), dev(idx), scale)
-    assert_attn_close(host(out), want, "out", sharp=scale > 4.0)
+    assert_attn_close(host(out), want, "out", sharp=scale > 4.0,
+                      vmax=row_vmax(oracle.fp4_kv_unpack(packed, sc), idx))
     assert_lse_close(host(lse), want_lse, "lse")
     assert np.all(host(out)[0, 0] == 0.0)
+
+
+def _block_case(seed, B, N, K, magnitude):
+    """Block-layout caches at the value ranges the pages report and below:
+    'pages' scales every (64-entry block, channel) to a maximum between 10 and
+    22 ('Detailed Notes On DeepSeek V4 Point 1 Flash In Simple Words', section
+    'FP4 Main KV Cache To Halve Storage Again': observed maxima of about 10 to
+    22, so no global scale is needed); 'subnormal' makes every block maximum below
+    0.075, so scale = max / 6 rounds to a nonzero E4M3 subnormal (1 to 7
+    times 2^-9)."""
+    rng = np.random.default_rng(seed)
+    kv = rng.standard_normal((B, N, 512)).astype(np.float32)
+    blk = kv.reshape(B, N // 64, 64, 512)
+    amax = np.abs(blk).max(axis=2, keepdims=True)
+    if magnitude == "pages":
+        target = rng.uniform(10.0, 22.0, amax.shape).astype(np.float32)
+    else:
+        target = rng.uniform(0.012, 0.075, amax.shape).astype(np.float32)
+    kv = (blk / amax * target).reshape(B, N, 512).astype(np.float32)
+    packed, scale = oracle.fp4_kv_pack(kv)
+    if magnitude == "subnormal":
+        assert np.all((scale & 0x78) == 0) and np.all(scale != 0), "nonzero subnormal scales"
+    idx = np.stack([np.sort(rng.choice(N, K, replace=False)) for _ in range(B)])[:, None, :]
+    return packed, scale, idx.astype(np.int32)
+
+
+# the in-cluster merge (2 rows, 4 splits) and the combine kernel (3 rows, 32 splits)
+@pytest.mark.parametrize("B,N,K", [(2, 4096, 256), (3, 16384, 2048)])
+@pytest.mark.parametrize("magnitude", ["pages", "subnormal"])
+@pytest.mark.parametrize("scale", [1.0 / math.sqrt(512.0), 1.0])
+def test_sparse_attn_block_layout_value_ranges(B, N, K, magnitude, scale):
+    packed, sc, idx = _block_case(B * 31 + K, B, N, K, magnitude)
+    rng = np.random.default_rng(B + K)
+    q = wl._to_bf16_bits(rng.standard_normal((B, 1, 64, 512)).astype(np.float32) / math.sqrt(512))
+    want, want_lse = oracle.sparse_attn(q, packed, sc, idx, scale)
+    out, lse = csa2.csa2_sparse_attn(bf16_dev(q), dev(packed), dev(sc), dev(idx), scale)
+    csa2.check_device_errors()
+    assert_attn_close(host(out), want, "out %s" % magnitude, sharp=True,
+                      vmax=row_vmax(oracle.fp4_kv_unpack(packed, sc), idx))
+    assert_lse_close(host(lse), want_lse, "lse %s" % magnitude)
 
 
 def test_sparse_attn_rising_max_across_tiles():
@@ -218,10 +260,11 @@ def test_sparse_attn_rising_max_across_tiles():
         order = np.argsort(logits[0])                  # head 0: ascending logit
         idx[b, 0] = np.sort(order[-K:]).astype(np.int32)
         idx[b, 0] = order[-K:].astype(np.int32)        # unsorted: rising logits along the list
+    vmax = row_vmax(V, idx)
     for scale in (8.0, 40.0):
         want, want_lse = oracle.sparse_attn(q, packed, sc, idx, scale)
         out, lse = csa2.csa2_sparse_attn(bf16_dev(q), dev(packed), dev(sc), dev(idx), scale)
-        assert_attn_close(host(out), want, "out scale=%g" % scale, sharp=True)
+        assert_attn_close(host(out), want, "out scale=%g" % scale, sharp=True, vmax=vmax)
         assert_lse_close(host(lse), want_lse, "lse scale=%g" % scale)
 
 
