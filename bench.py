@@ -447,6 +447,8 @@ def run_ours(args):
     if w.name == DEFAULT_WORKLOAD:
         line["attn_kv_g16"] = g16_attention(args, w, dw, csa2, torch, flush_l2, stream, acc0,
                                             peaks)
+        line["attn_kv_swa"] = swa_attention(args, w, dw, csa2, wl, torch, flush_l2, stream,
+                                            acc0, peaks, kern_us["attn"])
         if not args.no_prefill:
             line["prefill_indexer"] = prefill_indexer(args, dev, csa2, torch, flush_l2, stream,
                                                       peaks)
@@ -599,6 +601,48 @@ def g16_attention(args, w, dw, csa2, torch, flush_l2, stream, acc, peaks):
             "attn_us": us, "algorithmic_bytes": byts, "gbs": gbs,
             "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
             "cache": "the step's block-scaled cache dequantised and re-quantised per 16 channels"}
+
+
+def swa_attention(args, w, dw, csa2, wl, torch, flush_l2, stream, acc, peaks, attn_us):
+    """The attention kernel with the sliding-window branch: the step's queries,
+    cache and top-K plus each row's full window of 128 E4M3 tokens, one
+    softmax over both, timed like the per-kernel times (L2 flushed before each
+    call, device events). The window adds 128 rows of 512 bytes per query row
+    to the bytes read and 128 entries to each row's list."""
+    swa = torch.from_numpy(wl.swa_kv(w)).to(dw.kv_packed.device)
+    swa_n = torch.from_numpy(wl.swa_n(w)).to(dw.kv_packed.device)
+    out = torch.empty_like(dw.out[0])
+    lse = torch.empty_like(dw.lse[0])
+    W = wl.SWA_WINDOW
+    need = csa2.load().csa2_sparse_attn_workspace_bytes(w.B, w.Tq, w.Hq, w.D, w.K + W)
+    ws = torch.empty(max(int(need), 256), dtype=torch.uint8, device=swa.device)
+    times = []
+    for i in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush_l2(i)
+        e0.record(stream)
+        csa2.csa2_sparse_attn_swa(dw.q[0], dw.kv_packed, dw.kv_scale, dw.topk, swa, swa_n,
+                                  w.softmax_scale, W=W, out=out, lse=lse, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    csa2.check_device_errors()
+    us = 1e3 * statistics.mean(times)
+    rows_q = w.B * w.Tq
+    win_tokens = int(np.minimum(wl.swa_n(w), W).sum())
+    win_bytes = win_tokens * w.D
+    byts = acc["attn"] + win_bytes
+    flops = acc["attn_flops"] + win_tokens * w.Hq * w.D * 4
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"window": W, "window_format": "E4M3, one 512-byte row per token, no scale",
+            "combine": "one softmax over the selected rows and the window",
+            "attn_us": us, "attn_us_without_window": attn_us,
+            "window_tokens": win_tokens, "window_bytes": win_bytes,
+            "algorithmic_bytes": byts, "flops": flops, "gbs": gbs,
+            "frac_of_measured_hbm": gbs / peaks["hbm_gbs"],
+            "tflops": flops / (us * 1e-6) / 1e12,
+            "query_rows": rows_q}
 
 
 def run_e2e(args, w, dw, csa2, torch):

@@ -42,7 +42,8 @@ class LayerArgs(ctypes.Structure):
                 ("q", ctypes.c_void_p), ("idx_q", ctypes.c_void_p), ("idx_w", ctypes.c_void_p),
                 ("softmax_scale", ctypes.c_float), ("out", ctypes.c_void_p),
                 ("lse", ctypes.c_void_p), ("emit_pool", ctypes.c_int),
-                ("use_pool", ctypes.c_int)]
+                ("use_pool", ctypes.c_int), ("swa_kv", ctypes.c_void_p),
+                ("swa_n", ctypes.c_void_p), ("Tw", ctypes.c_int), ("W", ctypes.c_int)]
 
 
 EXPORTS = ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk",
@@ -50,7 +51,7 @@ EXPORTS = ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk",
            "csa2_layer_step_workspace_bytes", "csa2_layer_step", "csa2_check_device_errors",
            "csa2_last_error", "csa2_sparse_attn_noalloc", "fp4_kv_pack_g16", "fp4_kv_unpack_g16",
            "fp4_kv_append_g16", "csa2_sparse_attn_g16", "csa2_block_pool_workspace_bytes",
-           "csa2_block_pool")
+           "csa2_block_pool", "csa2_sparse_attn_swa")
 
 _lib = None
 
@@ -77,6 +78,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fp4_kv_unpack_g16.argtypes = [P, I, I, I, P, P]
     L.fp4_kv_append_g16.argtypes = [P, P, I, I, I, I, P, P]
     L.csa2_sparse_attn_g16.argtypes = [P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
+    L.csa2_sparse_attn_swa.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, Z,
+                                       P]
     L.csa2_block_pool_workspace_bytes.argtypes = [I, I, I, I, I]
     L.csa2_block_pool_workspace_bytes.restype = Z
     L.csa2_block_pool.argtypes = [P, I, P, I, I, I, I, P, P, Z, P]
@@ -90,7 +93,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for f in ("fp4_kv_pack", "fp4_kv_unpack", "csa2_index_score", "csa2_topk", "csa2_sparse_attn",
               "csa2_layer_step", "csa2_check_device_errors", "csa2_sparse_attn_noalloc",
               "fp4_kv_pack_g16", "fp4_kv_unpack_g16", "fp4_kv_append_g16", "csa2_sparse_attn_g16",
-              "csa2_block_pool"):
+              "csa2_block_pool", "csa2_sparse_attn_swa"):
         getattr(L, f).restype = I
     _lib = L
     return L
@@ -304,6 +307,43 @@ def csa2_sparse_attn_g16(q: torch.Tensor, kv_rows: torch.Tensor, topk_idx: torch
     return out, (lse if want_lse else None)
 
 
+SWA_WINDOW = 128   # tokens in the sliding window of every CSA2 layer
+
+
+def csa2_sparse_attn_swa(q: torch.Tensor, kv_packed: torch.Tensor,
+                         kv_scale: Optional[torch.Tensor], topk_idx: torch.Tensor,
+                         swa_kv: torch.Tensor, swa_n: torch.Tensor, softmax_scale: float,
+                         W: int = SWA_WINDOW, want_lse: bool = True,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None):
+    """csa2_sparse_attn plus the sliding-window branch: one softmax over the
+    selected rows and the tokens [max(0, n - W), n) of each row's E4M3 window
+    memory swa_kv uint8 [B][Tw][D], n = swa_n int32 [B][Tq]. kv_scale None:
+    kv_packed is in the 16-channel layout."""
+    _want(q, torch.bfloat16, "q", 4)
+    _want(topk_idx, torch.int32, "topk_idx", 3)
+    _want(swa_kv, torch.uint8, "swa_kv", 3)
+    _want(swa_n, torch.int32, "swa_n", 2)
+    B, Tq, Hq, D = q.shape
+    N = kv_packed.shape[1]
+    K = topk_idx.shape[-1]
+    Tw = swa_kv.shape[1]
+    L = load()
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Tq, Hq), dtype=torch.float32, device=q.device)
+    need = L.csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K + int(W))
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(L.csa2_sparse_attn_swa(_p(q), _p(kv_packed), _p(kv_scale), _p(topk_idx), _p(swa_kv),
+                                  _p(swa_n), B, Tq, Hq, D, N, K, Tw, int(W),
+                                  float(softmax_scale), _p(out), _p(lse if want_lse else None),
+                                  _p(workspace) if need else None, need, _stream(q.device)),
+           "csa2_sparse_attn_swa")
+    return out, (lse if want_lse else None)
+
+
 def csa2_sparse_attn_noalloc(q: torch.Tensor, kv_packed: torch.Tensor, kv_scale: torch.Tensor,
                              topk_idx: torch.Tensor, softmax_scale: float, want_lse: bool = True,
                              out: Optional[torch.Tensor] = None,
@@ -342,15 +382,19 @@ class Csa2Shared:
 
 
 def layer_args(q, nvalid, out, K, softmax_scale, idx_q=None, idx_w=None, lse=None, N=None,
-               emit_pool=False, use_pool=False) -> LayerArgs:
-    """emit_pool: False/0 none, True/1 the top-C entries, 2 the blockwise pool."""
+               emit_pool=False, use_pool=False, swa_kv=None, swa_n=None,
+               W=SWA_WINDOW) -> LayerArgs:
+    """emit_pool: False/0 none, True/1 the top-C entries, 2 the blockwise pool.
+    swa_kv / swa_n: the sliding-window branch (as in csa2_sparse_attn_swa)."""
     B, Tq, Hq, D = q.shape
     Hi = Di = 0
     if idx_q is not None:
         Hi, Di = idx_q.shape[2], idx_q.shape[3]
+    Tw = 0 if swa_kv is None else int(swa_kv.shape[1])
     return LayerArgs(B, Tq, int(N), D, Hq, Hi, Di, int(K), _p(nvalid), _p(q), _p(idx_q),
                      _p(idx_w), float(softmax_scale), _p(out), _p(lse), int(emit_pool),
-                     int(bool(use_pool)))
+                     int(bool(use_pool)), _p(swa_kv), _p(swa_n), Tw,
+                     int(W) if swa_kv is not None else 0)
 
 
 def csa2_layer_step(mode, args: LayerArgs, shared: Csa2Shared,

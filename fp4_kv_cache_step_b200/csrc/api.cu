@@ -301,12 +301,16 @@ csa2_status csa2_sparse_attn(const uint16_t* q, const uint8_t* kv_packed, const 
                              size_t workspace_bytes, csa2_stream_t stream) {
   csa2_status s = check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
   if (s != CSA2_OK) return s;
+  // the workspace is sized on the stream's device, as the launch plans it
+  // (with no device at all, for 148 SMs, so that the check still runs)
+  csa2::DeviceScope scope;
+  const cudaError_t se = scope.enter((cudaStream_t)stream);
   const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
     return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn needs %zu workspace bytes (got %zu)", need,
                 workspace_bytes);
+  if (se != cudaSuccess) return cuda_fail(se, "csa2_sparse_attn device");
   cudaError_t e;
-  csa2::DeviceScope scope;
   int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_sparse_attn");
   e = csa2::launch_sparse_attn(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, N, K, softmax_scale,
@@ -321,18 +325,60 @@ csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_rows,
                                  void* workspace, size_t workspace_bytes, csa2_stream_t stream) {
   csa2_status s = check_attn_any(q, kv_rows, nullptr, topk_idx, B, Tq, Hq, D, N, K, out, lse);
   if (s != CSA2_OK) return s;
+  csa2::DeviceScope scope;
+  const cudaError_t se = scope.enter((cudaStream_t)stream);
   const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
     return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn_g16 needs %zu workspace bytes (got %zu)",
                 need, workspace_bytes);
+  if (se != cudaSuccess) return cuda_fail(se, "csa2_sparse_attn_g16 device");
   cudaError_t e;
-  csa2::DeviceScope scope;
   int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_sparse_attn_g16");
   // a NULL block-scale array selects the 16-channel layout
   e = csa2::launch_sparse_attn(q, kv_rows, nullptr, topk_idx, B, Tq, Hq, N, K, softmax_scale, out,
                                lse, workspace, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "csa2_sparse_attn_g16 launch");
+  return ok();
+}
+
+namespace {
+csa2_status check_swa_args(const uint8_t* swa_kv, const int32_t* swa_n, int B, int Tw, int W,
+                           int K) {
+  CHECK_PTR(swa_kv);
+  CHECK_ARG(swa_n != nullptr && ((uintptr_t)swa_n & 3u) == 0,
+            "swa_n must be a non-null 4-byte aligned device pointer");
+  CHECK_ARG(Tw >= 0 && (size_t)B * Tw <= ((size_t)1 << 40), "Tw=%d must be >= 0", Tw);
+  CHECK_ARG(W >= 0 && W <= 65536, "W=%d must be in [0, 65536]", W);
+  CHECK_ARG((long long)K + W <= ((long long)1 << 30), "K + W must be <= 2^30");
+  return CSA2_OK;
+}
+}  // namespace
+
+csa2_status csa2_sparse_attn_swa(const uint16_t* q, const uint8_t* kv_packed,
+                                 const uint8_t* kv_scale, const int32_t* topk_idx,
+                                 const uint8_t* swa_kv, const int32_t* swa_n, int B, int Tq, int Hq,
+                                 int D, int N, int K, int Tw, int W, float softmax_scale,
+                                 uint16_t* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, csa2_stream_t stream) {
+  csa2_status s = check_attn_any(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K, out, lse);
+  if (s != CSA2_OK) return s;
+  s = check_swa_args(swa_kv, swa_n, B, Tw, W, K);
+  if (s != CSA2_OK) return s;
+  csa2::DeviceScope scope;
+  const cudaError_t se = scope.enter((cudaStream_t)stream);
+  const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K + W);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA2_ERR_WORKSPACE, "csa2_sparse_attn_swa needs %zu workspace bytes (got %zu)",
+                need, workspace_bytes);
+  if (se != cudaSuccess) return cuda_fail(se, "csa2_sparse_attn_swa device");
+  cudaError_t e;
+  int* err = device_error_word((cudaStream_t)stream, scope, &e);
+  if (!err) return cuda_fail(e, "csa2_sparse_attn_swa");
+  const csa2::SwaWindow win{swa_kv, swa_n, Tw, W};
+  e = csa2::launch_sparse_attn(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, N, K, softmax_scale,
+                               out, lse, workspace, err, (cudaStream_t)stream, &win);
+  if (e != cudaSuccess) return cuda_fail(e, "csa2_sparse_attn_swa launch");
   return ok();
 }
 
@@ -378,8 +424,10 @@ static size_t layer_pool_bytes(const csa2_layer_args* a, csa2_mode mode,
 size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* a, csa2_mode mode,
                                        const csa2_shared_state* st) {
   if (!a || !st) return 0;
+  // with a window, its W slots follow the K selected entries
+  const int W = a->swa_kv ? a->W : 0;
   return layer_scores_bytes(a, mode, st) + layer_pool_bytes(a, mode, st) +
-         csa2_sparse_attn_workspace_bytes(a->B, a->Tq, a->Hq, a->D, a->K);
+         csa2_sparse_attn_workspace_bytes(a->B, a->Tq, a->Hq, a->D, a->K + W);
 }
 
 csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_shared_state* st,
@@ -411,12 +459,18 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
       CHECK_ARG(st->C % kPoolBlock == 0 && st->C / kPoolBlock >= a->K,
                 "a blockwise pool needs C=%d a multiple of 8 with C/8 >= K=%d", st->C, a->K);
   }
+  if (a->swa_kv) {
+    s = check_swa_args(a->swa_kv, a->swa_n, a->B, a->Tw, a->W, a->K);
+    if (s != CSA2_OK) return s;
+  }
+  csa2::DeviceScope scope;
+  const cudaError_t se = scope.enter((cudaStream_t)stream);
   const size_t need = csa2_layer_step_workspace_bytes(a, mode, st);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
     return fail(CSA2_ERR_WORKSPACE, "csa2_layer_step needs %zu workspace bytes (got %zu)", need,
                 workspace_bytes);
+  if (se != cudaSuccess) return cuda_fail(se, "csa2_layer_step device");
   cudaError_t e;
-  csa2::DeviceScope scope;
   int* err = device_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return cuda_fail(e, "csa2_layer_step");
   cudaStream_t cs = (cudaStream_t)stream;
@@ -441,9 +495,11 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
       if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step block pool");
     }
   }
+  const csa2::SwaWindow win{a->swa_kv, a->swa_n, a->Tw, a->W};
   e = csa2::launch_sparse_attn(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq, a->Hq,
                                a->N, a->K, a->softmax_scale, a->out, a->lse,
-                               ws ? ws + scores_bytes + pool_bytes : nullptr, err, cs);
+                               ws ? ws + scores_bytes + pool_bytes : nullptr, err, cs,
+                               a->swa_kv ? &win : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step attention");
   return ok();
 }

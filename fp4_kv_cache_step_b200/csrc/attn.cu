@@ -101,10 +101,12 @@ size_t sparse_attn_workspace_bytes(int B, int Tq, int Hq, int K) {
 cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
-                               float* lse, void* workspace, int* err, cudaStream_t stream) {
+                               float* lse, void* workspace, int* err, cudaStream_t stream,
+                               const SwaWindow* swa) {
   const int rows = B * Tq;
   if (rows == 0) return cudaSuccess;
-  SplitPlan p = plan_splits(rows, Hq, K);
+  // the window's entries follow the selected ones in each row's entry list
+  SplitPlan p = plan_splits(rows, Hq, K + (swa ? swa->W : 0));
   float* ws_o = nullptr;
   float2* ws_ml = nullptr;
   if (p.nsplit > 1) {
@@ -115,7 +117,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
   bool merged = false;
   cudaError_t e = launch_sparse_attn_tc(q, kv_packed, kv_scale, topk_idx, rows, Tq, Hq, N, K,
                                         softmax_scale, p.nhb, p.nsplit, p.split_len, out, lse,
-                                        ws_o, ws_ml, err, stream, &merged);
+                                        ws_o, ws_ml, err, stream, &merged, swa);
   if (e != cudaSuccess || p.nsplit == 1 || merged) return e;
   return launch_pdl(attn_combine_kernel, dim3(rows, Hq), dim3(128), 0, stream, dim3(1), ws_o,
                     ws_ml, Hq, p.nhb, p.nsplit, out, lse);

@@ -218,11 +218,31 @@ __device__ __forceinline__ uint4 dq8(uint32_t codes, uint32_t s_lo, uint32_t s_h
   return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
+// 8 E4M3 bytes (two words, the first byte lowest) -> one 16-byte chunk of
+// fp16 values, times 2^-8 like the FP4 chunks: byte b becomes
+// ((b & 0x7f) << 7) | ((b & 0x80) << 8). *nan gets a nonzero bit for each
+// E4M3 NaN (0x7f, 0xff), whose fp16 pattern 0x3f80 no finite E4M3 value has.
+__device__ __forceinline__ uint4 e4m3x8(uint32_t a, uint32_t b, uint32_t* nan) {
+  uint32_t h[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    // halfwords (byte << 8) of bytes 2 (j & 1) and 2 (j & 1) + 1 of the word
+    const uint32_t x = __byte_perm(j < 2 ? a : b, 0u, (j & 1) ? 0x3424u : 0x1404u);
+    h[j] = (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
+    *nan |= __vcmpeq2(h[j] & 0x7fff7fffu, 0x3f803f80u);
+  }
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
 struct AttnParams {
   const uint16_t* q;
   const uint8_t* kv_packed;     // codes [B][N][D/2]; or rows [B][N][D/2 + D/16] (16-channel scales)
   const uint8_t* kv_scale;      // block scales [B][N/64][D]; unused for the 16-channel layout
   const int32_t* topk;
+  const uint8_t* swa_kv;        // window memory [B][Tw][D] E4M3 (entries K .. Ktot-1), or null
+  const int32_t* swa_n;         // [B][Tq]: the window of row (b, t) ends before token swa_n
+  int Tw, W;
+  int Ktot;                     // K selected entries, then W window slots
   int Tq, Hq, N, K, split_len, nsplit, nhb;
   float softmax_scale;
   uint16_t* out;
@@ -234,10 +254,12 @@ struct AttnParams {
 };
 
 // Raw bytes a producer lane holds for one entry: the codes (8 B) and scales
-// (16 B) of dims 16u .. 16u+15 and of dims 256+16u .. 256+16u+15.
+// (16 B) of dims 16u .. 16u+15 and of dims 256+16u .. 256+16u+15; for a window
+// token (win), its E4M3 bytes of those dims in s[0] and s[1].
 struct Raw {
   uint2 c[2];
   uint4 s[2];
+  bool win;
 };
 
 // The columns of the O accumulator a warp writes out at the end: its quadrant's
@@ -276,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   const int h0 = hb * kHB;
   const int nh = min(kHB, p.Hq - h0);
   const int k_begin = split * p.split_len;
-  const int k_end = min(p.K, k_begin + p.split_len);
+  const int k_end = min(p.Ktot, k_begin + p.split_len);
   const int nt = (k_end - k_begin + kT - 1) / kT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -325,14 +347,32 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     const uint8_t* pk_b = p.kv_packed + (size_t)b * p.N * kRowBytes;
     const uint8_t* sc_b = kG16 ? nullptr : p.kv_scale + (size_t)b * (p.N / kBlockEntries) * kD;
     const int32_t* topk_row = p.topk + row * p.K;
+    // the row's window: tokens [w_lo, w_hi) of its window memory (an end
+    // outside [0, Tw] is recorded and leaves the window empty)
+    const uint8_t* swa_b = p.swa_kv ? p.swa_kv + (size_t)b * p.Tw * kD : nullptr;
+    int w_hi = 0, w_lo = 0;
+    if (p.swa_kv && p.Ktot > p.K) {
+      w_hi = __ldg(p.swa_n + row);
+      if (w_hi < 0 || w_hi > p.Tw) {
+        if (lane == 0 && warp == 0 && hb == 0 && split == 0) record_error(p.err, CSA2_ERR_DEVICE_INDEX);
+        w_hi = 0;
+      }
+      w_lo = max(0, w_hi - p.W);
+    }
 
     // lanes 0-7: index of entry 8w + lane of tile t, as loaded (checked later:
-    // the check waits for the load, so it runs a tile after the load was issued)
+    // the check waits for the load, so it runs a tile after the load was
+    // issued). Window slot s (entry K + s) is token w_lo + s, given as
+    // -2 - token, or -1 past the window's end.
     auto fetch_index = [&](int t) -> int {
       const int kk = k_begin + t * kT + warp * 8 + lane;
-      return (lane < 8 && t < nt && kk < k_end) ? __ldg(topk_row + kk) : -1;
+      if (lane >= 8 || t >= nt || kk >= k_end) return -1;
+      if (kk < p.K) return __ldg(topk_row + kk);
+      const int tok = w_lo + (kk - p.K);
+      return tok < w_hi ? -2 - tok : -1;
     };
-    auto check_index = [&](int id) -> int {
+    auto check_index = [&](int id, int t) -> int {
+      if (k_begin + t * kT + warp * 8 + lane >= p.K) return id;   // a window slot, not loaded
       if (id >= p.N || id < -1) {
         record_error(p.err, CSA2_ERR_DEVICE_INDEX);
         id = -1;
@@ -345,7 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     // cover it.
     auto prefetch_rows = [&](int ids) {
       const int id = __shfl_sync(0xffffffffu, ids, lane >> 2);
-      if (id >= 0) {
+      if (id <= -2) {
+        // a window token: its 512-byte E4M3 row, one line per lane
+        const uint8_t* wr = swa_b + (size_t)(-2 - id) * kD + (lane & 3) * 128;
+        asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wr));
+      } else if (id >= 0) {
         const int q = lane & 3;
         if (kG16) {
           if (q < 3) {
@@ -367,7 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int id = __shfl_sync(0xffffffffu, ids, 2 * (2 * hf + k) + half);
-        if (id >= 0) {
+        r[k].win = id <= -2;
+        if (id <= -2) {
+          const uint8_t* wr = swa_b + (size_t)(-2 - id) * kD + 16 * u;
+          r[k].s[0] = __ldg(reinterpret_cast<const uint4*>(wr));
+          r[k].s[1] = __ldg(reinterpret_cast<const uint4*>(wr + 256));
+        } else if (id >= 0) {
           const uint8_t* pr = pk_b + (size_t)id * kRowBytes + 8 * u;
           r[k].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
           r[k].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
@@ -391,12 +440,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     };
     auto dequant_half = [&](const Raw (&r)[2], uint4 (&d)[2][4]) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
+      for (int k = 0; k < 2; ++k) {
+        if (r[k].win) {
+          uint32_t nan = 0;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          d[k][2 * hh] = dq8(r[k].c[hh].x, r[k].s[hh].x, r[k].s[hh].y);
-          d[k][2 * hh + 1] = dq8(r[k].c[hh].y, r[k].s[hh].z, r[k].s[hh].w);
+          for (int hh = 0; hh < 2; ++hh) {
+            d[k][2 * hh] = e4m3x8(r[k].s[hh].x, r[k].s[hh].y, &nan);
+            d[k][2 * hh + 1] = e4m3x8(r[k].s[hh].z, r[k].s[hh].w, &nan);
+          }
+          if (nan) record_error(p.err, CSA2_ERR_NONFINITE);
+        } else {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            d[k][2 * hh] = dq8(r[k].c[hh].x, r[k].s[hh].x, r[k].s[hh].y);
+            d[k][2 * hh + 1] = dq8(r[k].c[hh].y, r[k].s[hh].z, r[k].s[hh].w);
+          }
         }
+      }
     };
     auto store_half = [&](uint32_t tile, const uint4 (&d)[2][4], int hf) {
 #pragma unroll
@@ -498,9 +558,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     // has landed), rows prefetched into L2 two tiles ahead, and the next tile's
     // raw bytes loaded while this tile is dequantised (half by half), so a
     // producer never waits for a load it has just issued.
-    int id_cur = check_index(fetch_index(0));
-    int id_next = check_index(fetch_index(1));
-    int id_after = check_index(fetch_index(2));
+    int id_cur = check_index(fetch_index(0), 0);
+    int id_next = check_index(fetch_index(1), 1);
+    int id_after = check_index(fetch_index(2), 2);
     int id_far = fetch_index(3);
     prefetch_rows(id_cur);
     prefetch_rows(id_next);
@@ -514,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       uint4 dq[2][4];
       dequant_half(ra, dq);
       load_half(id_next, ra, 0);
-      const uint32_t vb = __ballot_sync(0xffffffffu, id_cur >= 0);   // lanes 8-31 hold -1
+      const uint32_t vb = __ballot_sync(0xffffffffu, id_cur != -1);   // lanes 8-31 hold -1
       // the slot (and its valid bits) is free once P(t-3) V(t-3) has completed;
       // slot 2 first holds the query block until the softmax warps have read it
       if (!mbar_wait_warp(&sm.bar.v_free[buf], ((t / kRing) & 1) ^ 1, abort_flag)) break;
@@ -528,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.v_full[buf]);
-      const int id_far_checked = check_index(id_far);
+      const int id_far_checked = check_index(id_far, t + 3);
       prefetch_rows(id_far_checked);
       id_far = fetch_index(t + 4);
       id_cur = id_next;
@@ -926,12 +986,17 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
                                   float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
-                                  bool* merged) {
+                                  bool* merged, const SwaWindow* swa) {
   AttnParams p;
   p.q = q;
   p.kv_packed = kv_packed;
   p.kv_scale = kv_scale;
   p.topk = topk_idx;
+  p.swa_kv = swa ? swa->kv : nullptr;
+  p.swa_n = swa ? swa->n : nullptr;
+  p.Tw = swa ? swa->Tw : 0;
+  p.W = swa ? swa->W : 0;
+  p.Ktot = K + p.W;
   p.Tq = Tq;
   p.Hq = Hq;
   p.N = N;

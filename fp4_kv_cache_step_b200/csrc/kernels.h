@@ -41,7 +41,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Makes the device a stream belongs to current for the rest of an entry point
 // (restoring the caller's current device on exit), so that the error word, any
 // built-in scratch and every launch belong to the stream's device. The legacy
-// and per-thread default streams belong to the current device.
+// and per-thread default streams belong to the current device. Entering again
+// for the same stream changes nothing (the caller's device stays the one
+// restored).
 class DeviceScope {
  public:
   DeviceScope() = default;
@@ -120,14 +122,26 @@ cudaError_t launch_block_pool(const float* scores, int ld, const int32_t* nvalid
                               int block, int nblocks, int32_t* cand, void* workspace, int* err,
                               cudaStream_t stream);
 
+// The sliding-window branch (csa2_sparse_attn_swa): window memory kv
+// [B][Tw][D] E4M3, one row per token, serving as key and value; query row
+// (b, t) also attends tokens [max(0, n[b][t] - W), n[b][t]). The kernels treat
+// the window as W more entries after the K selected ones.
+struct SwaWindow {
+  const uint8_t* kv;
+  const int32_t* n;
+  int Tw, W;
+};
+
 // Sparse attention; see csa2_sparse_attn. With kv_scale NULL, kv_packed holds
 // the 16-channel layout (csa2_sparse_attn_g16): per entry D/2 code bytes then
-// D/16 E4M3 scale bytes.
+// D/16 E4M3 scale bytes. With swa non-null the window branch joins the same
+// softmax; the workspace is then sized for K + swa->W entries.
 size_t sparse_attn_workspace_bytes(int B, int Tq, int Hq, int K);
 cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
-                               float* lse, void* workspace, int* err, cudaStream_t stream);
+                               float* lse, void* workspace, int* err, cudaStream_t stream,
+                               const SwaWindow* swa = nullptr);
 
 // Tensor-core attention kernel (attn_tc.cu). With nsplit > 1 the splits are
 // merged inside the kernel (thread-block clusters, *merged set to true) when
@@ -140,6 +154,6 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
                                   float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
-                                  bool* merged);
+                                  bool* merged, const SwaWindow* swa = nullptr);
 
 }  // namespace csa2

@@ -78,6 +78,10 @@ csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* kv_packed
   csa2_status s = csa2::api_check_attn_args(q, kv_packed, kv_scale, topk_idx, B, Tq, Hq, D, N, K,
                                             out, lse);
   if (s != CSA2_OK) return s;
+  // the stream's device is current from here on: the split plan, and with it
+  // the scratch size, follows its SM count
+  csa2::DeviceScope scope;
+  const cudaError_t se = scope.enter((cudaStream_t)stream);
   const size_t need = csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K);
   if (need > kNoAllocScratchBytes) {
     std::string msg = "csa2_sparse_attn_noalloc: this shape needs " + std::to_string(need) +
@@ -86,8 +90,8 @@ csa2_status csa2_sparse_attn_noalloc(const uint16_t* q, const uint8_t* kv_packed
                       "; use csa2_sparse_attn with a caller workspace";
     return csa2::api_fail(CSA2_ERR_WORKSPACE, msg.c_str());
   }
+  if (se != cudaSuccess) return csa2::api_cuda_fail(se, "csa2_sparse_attn_noalloc device");
   cudaError_t e;
-  csa2::DeviceScope scope;   // the stream's device is current from here on
   int* err = csa2::api_error_word((cudaStream_t)stream, scope, &e);
   if (!err) return csa2::api_cuda_fail(e, "csa2_sparse_attn_noalloc");
   void* scratch = nullptr;

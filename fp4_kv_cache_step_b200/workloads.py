@@ -34,6 +34,12 @@ indexer 32 heads x 128, 64 query heads of 512.
 Values: main KV ~ N(0, 1) (quantised by the library), queries ~ N(0, 1)/sqrt(512)
 rounded to bf16, indexer queries and keys integers uniform in [-4, 4] stored
 as E4M3, head weights integers uniform in [1, 4].
+
+The sliding-window branch every CSA2 layer has beside the sparse set (window
+of 128 tokens, its cache kept at 8 bits): each layer's window memory holds
+the W - 1 tokens before the query block and the block's own Tq tokens, values
+~ N(0, 1) rounded to E4M3; query t of a row sees the W tokens ending at its
+own (which sits at W - 1 + t): window memory [t, t + W), so swa_n = W + t.
 """
 from __future__ import annotations
 
@@ -44,7 +50,8 @@ from typing import Optional, Tuple
 import numpy as np
 import torch
 
-TAG_KV, TAG_IDXK, TAG_Q, TAG_IDXQ, TAG_W, TAG_LEN = 1, 2, 3, 4, 5, 6
+TAG_KV, TAG_IDXK, TAG_Q, TAG_IDXQ, TAG_W, TAG_LEN, TAG_SWA = 1, 2, 3, 4, 5, 6, 7
+SWA_WINDOW = 128
 
 FULL, REINDEX, REUSE = "FULL", "REINDEX", "REUSE"
 
@@ -152,6 +159,24 @@ def nvalid(w: Workload) -> np.ndarray:
     raise ValueError(w.lengths)
 
 
+def swa_tokens(w: Workload) -> int:
+    """Tokens in each row's window memory: the W - 1 before the query block
+    and the block's Tq."""
+    return w.Tq + SWA_WINDOW - 1
+
+
+def swa_kv_row(w: Workload, layer: int, b: int) -> np.ndarray:
+    """Window memory of batch row b at a layer: E4M3 bytes [Tw][D], N(0, 1)."""
+    x = _rng(w.seed, TAG_SWA, layer, b).standard_normal((swa_tokens(w), w.D), dtype=np.float32)
+    return _to_e4m3_bytes(x)
+
+
+def swa_n(w: Workload) -> np.ndarray:
+    """End of each query's window in the window memory: int32 [B][Tq], W + t."""
+    t = np.arange(w.Tq, dtype=np.int32) + SWA_WINDOW
+    return np.broadcast_to(t, (w.B, w.Tq)).copy()
+
+
 # ------------------------------------------------------------ whole tensors
 def _stack(fn, rows, *args):
     first = fn(*args, rows[0])
@@ -180,6 +205,10 @@ def idx_q(w: Workload, layer: int = 0, rows=None) -> np.ndarray:
 
 def idx_w(w: Workload, layer: int = 0, rows=None) -> np.ndarray:
     return _stack(lambda b: idx_w_row(w, layer, b), list(range(w.B)) if rows is None else list(rows))
+
+
+def swa_kv(w: Workload, layer: int = 0, rows=None) -> np.ndarray:
+    return _stack(lambda b: swa_kv_row(w, layer, b), list(range(w.B)) if rows is None else list(rows))
 
 
 # ------------------------------------------------------------ the model's stack

@@ -256,6 +256,39 @@ CSA2_API csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_r
                                           csa2_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * csa2_sparse_attn_swa -- csa2_sparse_attn plus the sliding-window branch
+ * that every CSA2 layer has beside its selected entries ([N] "The Three Modes
+ * Full Reindex And Reuse" and "Model Setup Numbers Without Jargon": a window
+ * of the last 128 tokens; [N] "FP4 Main KV Cache To Halve Storage Again" and
+ * [M] 3.5: the window's cache stays at 8 bits). The pages do not say how the
+ * two branches combine; here one softmax runs over the union of the selected
+ * main-KV rows and the window's tokens, each window row (D E4M3 values, no
+ * scale) serving as key and value:
+ *     entries of row (b, t) = {v_k : topk_idx[b][t][k] >= 0}
+ *                           + {e4m3(swa_kv[b][j]) : max(0, n - W) <= j < n},
+ *     n = swa_n[b][t]; then out and lse as in csa2_sparse_attn.
+ * Same arguments as csa2_sparse_attn (with kv_scale NULL, kv_packed holds the
+ * 16-channel layout as in csa2_sparse_attn_g16), plus:
+ *   swa_kv   uint8 [B][Tw][D]  E4M3 window memory; 16-byte aligned
+ *   swa_n    int32 [B][Tq]     end of each query row's window, in [0, Tw];
+ *                              an end outside it is recorded
+ *                              (CSA2_ERR_DEVICE_INDEX) and empties that window
+ *   Tw       tokens in each row's window memory (>= 0)
+ *   W        window length (128 in the pages; 0 <= W <= 65536)
+ * An E4M3 NaN byte (0x7f, 0xff) in a window row that is read records
+ * CSA2_ERR_NONFINITE (the outputs of that query row are then unspecified).
+ * The workspace is csa2_sparse_attn_workspace_bytes(B, Tq, Hq, D, K + W):
+ * the window's W slots follow the K selected entries in each row's list.
+ * ------------------------------------------------------------------------ */
+CSA2_API csa2_status csa2_sparse_attn_swa(const uint16_t* q, const uint8_t* kv_packed,
+                                          const uint8_t* kv_scale, const int32_t* topk_idx,
+                                          const uint8_t* swa_kv, const int32_t* swa_n, int B,
+                                          int Tq, int Hq, int D, int N, int K, int Tw, int W,
+                                          float softmax_scale, uint16_t* out, float* lse,
+                                          void* workspace, size_t workspace_bytes,
+                                          csa2_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * csa2_sparse_attn_noalloc -- csa2_sparse_attn without a caller workspace.
  * (An interface addition of this library; the pages describe no such call.)
  *
@@ -271,7 +304,9 @@ CSA2_API csa2_status csa2_sparse_attn_g16(const uint16_t* q, const uint8_t* kv_r
  * library reserves it, whether or not this function is ever called.
  *  - Returns CSA2_ERR_WORKSPACE, launching nothing, when the shape needs more
  *    split scratch than the array holds (compare with
- *    csa2_sparse_attn_workspace_bytes()).
+ *    csa2_sparse_attn_workspace_bytes()). The split plan gives each SM at most
+ *    one (row, head block, split) slot of 131,584 bytes, so on a GPU with up to
+ *    255 SMs (a B200 has 148) no shape needs more than the array.
  *  - All calls on a device share the array: calls that overlap on the GPU
  *    (e.g. two streams at once) race. The array keeps the last call's contents;
  *    nothing in it needs to start at zero.
@@ -327,6 +362,11 @@ typedef struct {
   int emit_pool;              /* FULL: 0 no pool; 1 the top-C entries; 2 the blockwise
                                  pool (blocks of 8, C/8 blocks, C % 8 == 0) into st->cand_idx */
   int use_pool;               /* REINDEX: score only st->cand_idx */
+  /* The sliding-window branch (csa2_sparse_attn_swa), in every mode; swa_kv
+     NULL leaves it out. The workspace then grows by the window's W slots. */
+  const uint8_t* swa_kv;      /* [B][Tw][D] E4M3 window memory, or NULL */
+  const int32_t* swa_n;       /* [B][Tq] end of each query row's window */
+  int Tw, W;
 } csa2_layer_args;
 
 CSA2_API size_t csa2_layer_step_workspace_bytes(const csa2_layer_args* args, csa2_mode mode,

@@ -98,6 +98,58 @@ def test_workspace_is_checked_before_launch(lib):
     assert lib.csa2_sparse_attn_workspace_bytes(32, 1, 64, 512, 2048) >= 32 * 4 * 64 * 512 * 4
 
 
+def test_swa_arguments_are_checked(lib):
+    P, F = ctypes.c_void_p, ctypes.c_float(1.0)
+    a = P(256)
+    # no window memory, a negative window, a misaligned window end array
+    rc = lib.csa2_sparse_attn_swa(a, a, a, a, None, a, 1, 1, 16, 512, 64, 8, 128, 128, F, a,
+                                  None, None, 0, None)
+    assert _status(rc) == "INVALID_ARG" and b"swa_kv" in lib.csa2_last_error()
+    rc = lib.csa2_sparse_attn_swa(a, a, a, a, a, a, 1, 1, 16, 512, 64, 8, 128, -1, F, a, None,
+                                  None, 0, None)
+    assert _status(rc) == "INVALID_ARG"
+    rc = lib.csa2_sparse_attn_swa(a, a, a, a, a, P(258), 1, 1, 16, 512, 64, 8, 128, 128, F, a,
+                                  None, None, 0, None)
+    assert _status(rc) == "INVALID_ARG"
+    # the window's slots follow the K selected entries: 2 rows of 256 + 128
+    # entries split 6 ways where 256 alone split 4 ways
+    ws_k = lib.csa2_sparse_attn_workspace_bytes(2, 1, 64, 512, 256)
+    ws_kw = lib.csa2_sparse_attn_workspace_bytes(2, 1, 64, 512, 256 + 128)
+    assert ws_kw > ws_k > 0
+    rc = lib.csa2_sparse_attn_swa(a, a, a, a, a, a, 2, 1, 64, 512, 4096, 256, 300, 128, F, a,
+                                  None, a, ws_k, None)
+    assert _status(rc) == "WORKSPACE"
+
+
+def test_layer_args_struct_matches_the_header():
+    """The binding's ctypes mirror of csa2_layer_args has the C layout (size
+    and the offsets of the window fields), checked by compiling the header."""
+    import subprocess
+    import tempfile
+    src = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "csa2.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\n", sizeof(csa2_layer_args), offsetof(csa2_layer_args, swa_kv),
+         offsetof(csa2_layer_args, swa_n), offsetof(csa2_layer_args, Tw),
+         offsetof(csa2_layer_args, W));
+  return 0;
+}
+"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        with open(c, "w") as f:
+            f.write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I",
+                        "/usr/local/cuda/include", c, "-o", exe], check=True)
+        got = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                               check=True).stdout.split()]
+    L = csa2.LayerArgs
+    assert got == [ctypes.sizeof(L), L.swa_kv.offset, L.swa_n.offset, L.Tw.offset, L.W.offset]
+
+
 def test_layer_step_rejects_bad_mode_and_pool(lib):
     sh = csa2.SharedState(256, 256, 256, 256, None, 0)
     args = csa2.LayerArgs(1, 1, 4096, 512, 16, 4, 64, 256, 256, 256, 256, 256, 1.0, 256, None, 1, 0)
