@@ -57,6 +57,14 @@ KERNEL_SOURCES = {
     "score": ("score_tc.cu", "sm100.cuh", "common.cuh"),
     "topk": ("topk.cu", "common.cuh"),
     "attn": ("attn_tc.cu", "attn.cu", "sm100.cuh", "common.cuh"),
+    "block_pool": ("pool.cu", "topk.cu", "common.cuh"),
+}
+# the kernels' names as ncu lists them (regular expressions)
+KERNEL_NAMES = {
+    "score": r"index_score",
+    "topk": r"topk_(reg_|cluster_)?kernel",
+    "attn": r"sparse_attn_tc_kernel",
+    "block_pool": r"block_(max|expand)_kernel",
 }
 
 
@@ -130,6 +138,63 @@ def profiled_traffic(kernel: str, workload: str, units: float):
         return float(best["dram_bytes_per_launch"]) * units / float(best["units"]), \
             "ncu capture of %s scaled by units (%s)" % (best["workload"], best.get("unit_kind"))
     return None, "sources changed since the last ncu capture"
+
+
+_NCU_SCALE = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-3,
+              "usecond": 1.0, "msecond": 1e3, "second": 1e6}
+
+
+def record_ncu(csv_path: str, kernel: str, workload: str, command: str, units=None,
+               unit_kind=None, out_path: str = TRAFFIC_FILE) -> dict:
+    """Turn one ncu capture (--csv with dram__bytes_read.sum, dram__bytes_write.sum
+    and gpu__time_duration.sum) into the per-launch record that the roofline's
+    `traffic` reads: the launches of `kernel` in the file, their mean DRAM bytes
+    and duration, the sha1 of the kernel's sources now, the workload and the
+    command that made the capture. Replaces the record of the same kernel and
+    workload in `out_path`."""
+    import csv
+    import re
+    pat = re.compile(KERNEL_NAMES[kernel])
+    per = {}
+    with open(csv_path, newline="") as f:
+        lines = [l for l in f if l.startswith('"')]       # ncu's own log lines are not CSV
+    for row in csv.DictReader(lines):
+        if not pat.search(row.get("Kernel Name", "")):
+            continue
+        name = row["Metric Name"]
+        if name not in ("dram__bytes_read.sum", "dram__bytes_write.sum", "gpu__time_duration.sum"):
+            continue
+        v = float(row["Metric Value"].replace(",", "")) * _NCU_SCALE.get(row["Metric Unit"], 1.0)
+        per.setdefault(row["ID"], {})[name] = v
+    launches = [m for m in per.values() if len(m) == 3]
+    if not launches:
+        raise SystemExit("no complete %s launch in %s" % (kernel, csv_path))
+    n = len(launches)
+    rec = {"kernel": kernel, "sources_sha1": sources_sha1(kernel), "workload": workload,
+           "launches": n,
+           "dram_read_bytes_per_launch": sum(m["dram__bytes_read.sum"] for m in launches) / n,
+           "dram_write_bytes_per_launch": sum(m["dram__bytes_write.sum"] for m in launches) / n,
+           "duration_us_under_ncu": sum(m["gpu__time_duration.sum"] for m in launches) / n,
+           "command": command}
+    rec["dram_bytes_per_launch"] = rec["dram_read_bytes_per_launch"] + \
+        rec["dram_write_bytes_per_launch"]
+    if units is not None:
+        rec["units"], rec["unit_kind"] = float(units), unit_kind
+    try:
+        with open(out_path) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        doc = {}
+    doc.setdefault("about", "DRAM bytes per launch of each timed kernel from ncu (cold "
+                            "caches, serialised launches), with the sha1 of the kernel's sources "
+                            "when captured; written by bench.py --record-ncu")
+    caps = [r for r in doc.get("captures", [])
+            if not (r.get("kernel") == kernel and r.get("workload") == workload)]
+    doc["captures"] = caps + [rec]
+    with open(out_path, "w") as f:
+        json.dump(doc, f, indent=1)
+        f.write("\n")
+    return rec
 
 
 def measured_peaks():
@@ -441,9 +506,13 @@ def run_ours(args):
                          for l, m in enumerate(w.modes)]
     line["kernel_us"] = kern_us
     line["roofline"] = roof
-    line["kernel_rooflines"] = {k: {kk: v[kk] for kk in ("bound", "achieved", "unit", "frac",
-                                                         "hbm_frac")}
-                                for k, v in rl.items()}
+    line["kernel_rooflines"] = {}
+    for k, v in rl.items():
+        kr = {kk: v[kk] for kk in ("bound", "achieved", "unit", "frac", "hbm_frac",
+                                   "algorithmic_bytes")}
+        kr["traffic"], kr["traffic_source"] = profiled_traffic(
+            k, w.name, acc0["selected"] if k == "attn" else acc0["keys"])
+        line["kernel_rooflines"][k] = kr
     if w.name == DEFAULT_WORKLOAD:
         line["attn_kv_g16"] = g16_attention(args, w, dw, csa2, torch, flush_l2, stream, acc0,
                                             peaks)
@@ -968,7 +1037,16 @@ def main():
                     help="time the model's 38 CSA2 layers (one GPU) instead of the headline step")
     ap.add_argument("--context", type=int, default=131072, help="--stack: context in tokens")
     ap.add_argument("--batch", type=int, default=4, help="--stack: sequences")
+    ap.add_argument("--record-ncu", default=None, metavar="CSV",
+                    help="write the DRAM traffic of --kernel from an ncu CSV capture of "
+                         "--workload into profiles/kernel_traffic.json (no GPU needed)")
+    ap.add_argument("--kernel", default=None, choices=sorted(KERNEL_NAMES))
+    ap.add_argument("--ncu-command", default="", help="--record-ncu: the capture's command")
     args = ap.parse_args()
+    if args.record_ncu:
+        rec = record_ncu(args.record_ncu, args.kernel, args.workload, args.ncu_command)
+        print(json.dumps(rec))
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.stack is not None and args.impl == "ours":
