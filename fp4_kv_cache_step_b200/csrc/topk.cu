@@ -15,7 +15,8 @@
 // keys of that bin are ranked exactly against each other. A crowded threshold
 // bin (many equal scores) falls back to an MSB-first 8-bit radix select. The
 // selection is written in id order by a two-pass, ballot-based compaction.
-// Rows that fit are staged once in shared memory.
+// Rows that fit are staged once in shared memory. Rows of up to 32768 keys take
+// the register variant at the end of this file.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -714,6 +715,477 @@ topk_cluster_kernel(const float* __restrict__ scores, int ld, const int32_t* __r
   }
 }
 
+// ---------------------------------------------------------------------------
+// Register variant. A row is split over a cluster of CS CTAs (CS = 1, 2, 4 or
+// 8) of 512 threads; CTA r of the cluster covers positions r S .. r S + S - 1,
+// S = 512 KPT (KPT a multiple of 4, at most 64). Warp w of a CTA covers 32 KPT
+// consecutive positions of its slice; its lane l holds the 4-key chunks at
+// w 32 KPT + 128 j + 4 l (j < KPT / 4), so every warp load is one coalesced
+// 512-byte line set, and after that single pass over the scores every step
+// works on registers and a few kilobytes of shared memory:
+//   1. keys, their count and range [kmin, kmax] (block reductions, then the
+//      cluster's ranges combined over distributed shared memory);
+//   2. a 4096-bin histogram over that range per CTA (shared-memory atomics),
+//      summed over the cluster, and a suffix scan to the bin holding the k-th
+//      key; a crowded bin is refined with the next 12 bits of the key, down to
+//      the key itself;
+//   3. the few keys of the threshold bin, gathered from the cluster, ranked
+//      exactly (score desc, index asc);
+//   4. the ordered write: each CTA's (greater, equal) counts give the offset
+//      of its slice, a block scan the offset of each warp, and per chunk row a
+//      warp scan the slot of each lane's keys.
+// Same ranking and output as the kernels above.
+
+constexpr int kRThreads = 512;
+constexpr int kRWarps = kRThreads / 32;
+constexpr int kRBins = 4096;
+constexpr int kRBinsPerThread = kRBins / kRThreads;
+constexpr int kRCandCap = 1024;
+
+struct __align__(16) RegShared {
+  int bins[kRBins];                 // this CTA's histogram (read by the cluster)
+  uint32_t cand_key[kRCandCap];     // this CTA's keys in the threshold bin (read by the cluster)
+  int cand_pos[kRCandCap];
+  uint32_t all_key[kRCandCap];      // the whole row's threshold bin
+  int all_pos[kRCandCap];
+  int warp_a[kRWarps], warp_b[kRWarps];
+  uint32_t red_min[kRWarps], red_max[kRWarps];
+  int bcast[4];
+  int ncand;
+  uint32_t loc_min, loc_max;        // this CTA's key range and count (read by the cluster)
+  int loc_cnt;
+  uint32_t loc_emit;                // this CTA's (greater << 16 | equal) counts (read by the cluster)
+};
+
+template <int CS>
+__device__ __forceinline__ void csync(cg::cluster_group& cl) {
+  if (CS > 1) cl.sync(); else __syncthreads();
+}
+
+template <int CS, typename T>
+__device__ __forceinline__ T* at_rank(cg::cluster_group& cl, T* p, int r) {
+  return CS > 1 ? cl.map_shared_rank(p, r) : p;
+}
+
+// position in the row of key (chunk j, element q) of this thread
+template <int KPT>
+__device__ __forceinline__ int reg_pos(int base, int j, int q) {
+  return base + (int)(threadIdx.x >> 5) * 32 * KPT + 128 * j + 4 * (int)(threadIdx.x & 31) + q;
+}
+
+// Exclusive prefix sum of v over the block (thread order).
+__device__ __forceinline__ int reg_block_scan(int v, int& total, RegShared& sc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sc.warp_a[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = lane < kRWarps ? sc.warp_a[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    if (lane < kRWarps) sc.warp_b[lane] = wi - w;
+    if (lane == 31) sc.bcast[3] = wi;
+  }
+  __syncthreads();
+  const int res = sc.warp_b[warp] + incl - v;
+  total = sc.bcast[3];
+  __syncthreads();
+  return res;
+}
+
+// (T, need_eq) of the k-th largest real key of the row (1 <= k <= its real
+// keys): T is the key, need_eq how many keys equal to T the selection takes.
+// `reads_pending`: the cluster may still read this CTA's histogram or
+// candidates from an earlier call.
+template <int KPT, int CS>
+__device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT], int base,
+                              uint32_t kmin, uint32_t kmax, int k, bool reads_pending,
+                              uint32_t& T, int& need_eq, RegShared& sc) {
+  uint32_t lo = kmin;
+  uint32_t width_m1 = kmax - kmin;                 // range [lo, lo + width_m1]
+  const int bits = width_m1 == 0u ? 0 : 32 - __clz(width_m1);
+  int shift = bits > 12 ? bits - 12 : 0;
+  int krem = k;
+  bool first = true;
+  for (;;) {
+    if (CS > 1 && (reads_pending || !first)) cl.sync();   // nobody still reads our histogram
+    for (int i = threadIdx.x; i < kRBins; i += kRThreads) sc.bins[i] = 0;
+    if (threadIdx.x == 0) sc.ncand = 0;
+    __syncthreads();
+    if (first) {
+      // every real key lies in the range
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if (key[j] != 0u) atomicAdd(&sc.bins[(key[j] - lo) >> shift], 1);
+    } else {
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t kk = key[j];
+        if (kk != 0u && kk >= lo && kk - lo <= width_m1) atomicAdd(&sc.bins[(kk - lo) >> shift], 1);
+      }
+    }
+    first = false;
+    csync<CS>(cl);                                 // the cluster's histograms are complete
+    // descending bins: thread t owns bins 4095 - 8t .. 4088 - 8t, summed over the cluster
+    const int b0 = kRBins - kRBinsPerThread * ((int)threadIdx.x + 1);
+    int loc[kRBinsPerThread] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int r = 0; r < CS; ++r) {
+      const int4* src = reinterpret_cast<const int4*>(at_rank<CS>(cl, sc.bins, r) + b0);
+      const int4 x = src[0], y = src[1];
+      loc[0] += y.w;
+      loc[1] += y.z;
+      loc[2] += y.y;
+      loc[3] += y.x;
+      loc[4] += x.w;
+      loc[5] += x.z;
+      loc[6] += x.y;
+      loc[7] += x.x;
+    }
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < kRBinsPerThread; ++j) mine += loc[j];
+    int tot;
+    int above = reg_block_scan(mine, tot, sc);
+    if (above < krem && krem <= above + mine) {
+#pragma unroll
+      for (int j = 0; j < kRBinsPerThread; ++j) {
+        if (above < krem && krem <= above + loc[j]) {
+          sc.bcast[0] = kRBins - 1 - kRBinsPerThread * (int)threadIdx.x - j;
+          sc.bcast[1] = krem - above;
+          sc.bcast[2] = loc[j];
+        }
+        above += loc[j];
+      }
+    }
+    __syncthreads();
+    const uint32_t bstar = (uint32_t)sc.bcast[0];
+    krem = sc.bcast[1];
+    const int cbin = sc.bcast[2];
+    lo += bstar << shift;
+    if (shift == 0) {
+      // the bin is a single key value
+      T = lo;
+      need_eq = krem;
+      __syncthreads();
+      return;
+    }
+    const uint32_t bw_m1 = (1u << shift) - 1u;
+    if (cbin <= kRCandCap) {
+      // the keys of the threshold bin, from the whole cluster, ranked exactly
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t kk = key[j];
+        if (kk != 0u && kk >= lo && kk - lo <= bw_m1) {
+          const int slot = atomicAdd(&sc.ncand, 1);
+          if (slot < kRCandCap) {
+            sc.cand_key[slot] = kk;
+            sc.cand_pos[slot] = reg_pos<KPT>(base, j / 4, j % 4);
+          }
+        }
+      }
+      csync<CS>(cl);                               // every CTA's candidates are listed
+      int c;
+      const uint32_t* ck = sc.cand_key;
+      const int* cp = sc.cand_pos;
+      if (CS > 1) {
+        int off = 0;
+        for (int r = 0; r < CS; ++r) {
+          RegShared* o = at_rank<CS>(cl, &sc, r);
+          const int nr = min(o->ncand, kRCandCap);
+          for (int u = threadIdx.x; u < nr; u += kRThreads) {
+            if (off + u < kRCandCap) {
+              sc.all_key[off + u] = o->cand_key[u];
+              sc.all_pos[off + u] = o->cand_pos[u];
+            }
+          }
+          off += nr;
+        }
+        c = min(off, kRCandCap);
+        ck = sc.all_key;
+        cp = sc.all_pos;
+        __syncthreads();
+      } else {
+        c = min(sc.ncand, kRCandCap);
+      }
+      for (int u = threadIdx.x; u < c; u += kRThreads) {
+        const uint32_t ku = ck[u];
+        const int pu = cp[u];
+        int gt = 0, eqb = 0;
+        for (int v = 0; v < c; ++v) {
+          const uint32_t kv = ck[v];
+          gt += kv > ku;
+          eqb += (kv == ku) && (cp[v] < pu);
+        }
+        if (gt + eqb == krem - 1) {
+          sc.bcast[0] = (int)ku;
+          sc.bcast[1] = eqb + 1;
+        }
+      }
+      __syncthreads();
+      T = (uint32_t)sc.bcast[0];
+      need_eq = sc.bcast[1];
+      __syncthreads();
+      return;
+    }
+    // crowded bin: the next 12 bits within it
+    width_m1 = bw_m1;
+    shift = shift > 12 ? shift - 12 : 0;
+    __syncthreads();
+  }
+}
+
+// Writes, in position order, every key above T and the first need_eq keys equal
+// to T (T = 0 selects every real key), then pads with -1 up to k.
+template <int KPT, int CS>
+__device__ void reg_emit(cg::cluster_group& cl, int rank, const uint32_t (&key)[KPT], int base,
+                         uint32_t T, int need_eq, int k, int n_valid, const int32_t* crow,
+                         int32_t* out, RegShared& sc) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // (greater << 16 | equal) counts: a CTA's totals (at most 512 x 64) fit 16 bits each
+  uint32_t c = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) c += ((uint32_t)(key[j] > T) << 16) | (uint32_t)(key[j] == T && key[j] != 0u);
+  const uint32_t wc = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) sc.warp_a[warp] = (int)wc;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = lane < kRWarps ? (uint32_t)sc.warp_a[lane] : 0u;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane < kRWarps) sc.warp_b[lane] = (int)(incl - v);
+    if (lane == 31) sc.loc_emit = incl;
+  }
+  csync<CS>(cl);                                   // every CTA's counts are published
+  // selected before this warp's first chunk row: the earlier CTAs' and warps'
+  int gt_run = 0, eq_run = 0;
+  for (int r = 0; r < rank; ++r) {
+    const uint32_t e = at_rank<CS>(cl, &sc, r)->loc_emit;
+    gt_run += (int)(e >> 16);
+    eq_run += (int)(e & 0xffffu);
+  }
+  gt_run += (int)((uint32_t)sc.warp_b[warp] >> 16);
+  eq_run += (int)((uint32_t)sc.warp_b[warp] & 0xffffu);
+#pragma unroll
+  for (int j = 0; j < KPT / 4; ++j) {
+    uint32_t cj = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      cj += ((uint32_t)(key[4 * j + q] > T) << 16) |
+            (uint32_t)(key[4 * j + q] == T && key[4 * j + q] != 0u);
+    uint32_t incl = cj;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t ex = incl - cj;
+    int eq_seen = eq_run + (int)(ex & 0xffffu);
+    int pos = gt_run + (int)(ex >> 16) + min(eq_seen, need_eq);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t kk = key[4 * j + q];
+      bool take = kk > T;
+      if (kk == T && kk != 0u) take = eq_seen++ < need_eq;
+      if (take) {
+        const int i = reg_pos<KPT>(base, j, q);
+        out[pos++] = crow ? __ldg(crow + i) : i;
+      }
+    }
+    gt_run += (int)(tot >> 16);
+    eq_run += (int)(tot & 0xffffu);
+  }
+  if (rank == CS - 1) {
+    const int total = min(k, n_valid);
+    for (int i = total + threadIdx.x; i < k; i += kRThreads) out[i] = -1;
+  }
+  __syncthreads();
+}
+
+template <int KPT, int CS, bool kPool>
+__global__ void __launch_bounds__(kRThreads, 1)
+topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict__ nvalid,
+                const int32_t* __restrict__ cand, int K, int32_t* __restrict__ topk_out,
+                int Cout, int32_t* __restrict__ cand_out, int* err) {
+  static_assert(KPT % 4 == 0 && KPT <= 64, "chunks of four keys, at most 64 per thread");
+  __shared__ RegShared sc;
+  pdl_wait_and_release();
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = CS > 1 ? (int)cl.block_rank() : 0;
+  const size_t row = blockIdx.x / CS;
+  const int base = rank * kRThreads * KPT;          // first position of this CTA's slice
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* srow = scores + row * ld;
+  const int32_t* crow = kPool ? cand + row * ld : nullptr;
+  const int n = kPool ? ld : max(0, min(ld, nvalid[row]));
+  // Whole rows of 16-byte aligned, 4-key-divisible length take branch-free
+  // 16-byte loads (chunks past the row end read its first chunk, masked below),
+  // so all of a thread's loads are in flight together; other rows load keys one
+  // by one.
+  const bool vec = ld % 4 == 0 && ld >= 4 &&
+                   ((reinterpret_cast<uintptr_t>(srow) | reinterpret_cast<uintptr_t>(crow)) & 15u) == 0;
+  uint32_t key[KPT];
+  int ids[kPool ? KPT : 1];
+  if (vec) {
+#pragma unroll
+    for (int j = 0; j < KPT / 4; ++j) {
+      const int p0 = reg_pos<KPT>(base, j, 0);
+      const int pl = p0 < ld ? p0 : 0;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(srow + pl));
+      key[4 * j] = __float_as_uint(v.x);
+      key[4 * j + 1] = __float_as_uint(v.y);
+      key[4 * j + 2] = __float_as_uint(v.z);
+      key[4 * j + 3] = __float_as_uint(v.w);
+      if (kPool) {
+        const int4 cv = __ldg(reinterpret_cast<const int4*>(crow + pl));
+        ids[4 * j] = cv.x;
+        ids[4 * j + 1] = cv.y;
+        ids[4 * j + 2] = cv.z;
+        ids[4 * j + 3] = cv.w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int p = reg_pos<KPT>(base, j / 4, j % 4);
+      key[j] = p < n ? __float_as_uint(__ldg(srow + p)) : 0u;
+      if (kPool) ids[j] = p < n ? __ldg(crow + p) : -1;
+    }
+  }
+  uint64_t real = 0u;                  // bit 4 j + q: key (j, q) is a candidate
+  bool unsorted = false;
+  int prev_last = -1;                  // a pool's id at the position before the current chunk row
+#pragma unroll
+  for (int j = 0; j < KPT / 4; ++j) {
+    const int p0 = reg_pos<KPT>(base, j, 0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      real |= (uint64_t)((p0 + q < n && (!kPool || ids[4 * j + q] >= 0)) ? 1u : 0u) << (4 * j + q);
+    if (kPool) {
+      // ids ascending: each real id exceeds the id before it, which is real; the
+      // id before a chunk is the previous lane's last (lane 0: the last of lane
+      // 31 in the previous chunk row, or before the warp's first, from memory)
+      int prev = __shfl_up_sync(0xffffffffu, ids[4 * j + 3], 1);
+      if (lane == 0) prev = j > 0 ? prev_last : ((p0 > 0 && p0 - 1 < n) ? __ldg(crow + p0 - 1) : -1);
+      prev_last = __shfl_sync(0xffffffffu, ids[4 * j + 3], 31);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int id = ids[4 * j + q];
+        if (p0 + q < n && id >= 0 && p0 + q > 0 && (prev < 0 || prev >= id)) unsorted = true;
+        prev = id;
+      }
+    }
+  }
+  // order-preserving keys, branch-free: x ^ (sign ? ~0 : 0x80000000), -0 as +0,
+  // NaN and non-candidates 0 (a NaN is reported)
+  bool nan = false;
+  int mine = 0;
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const uint32_t u = key[j], a = u & 0x7fffffffu;
+    const bool is_real = (real >> j) & 1u;
+    const bool isnan = a > 0x7f800000u;
+    nan |= isnan && is_real;
+    uint32_t kk = a == 0u ? 0x80000000u : u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+    kk = (isnan || !is_real) ? 0u : kk;
+    key[j] = kk;
+    mine += kk != 0u;
+    kmin = min(kmin, kk == 0u ? 0xffffffffu : kk);
+    kmax = max(kmax, kk);
+  }
+  if (nan) record_error(err, CSA2_ERR_NONFINITE);
+  if (unsorted) record_error(err, CSA2_ERR_DEVICE_INDEX);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  mine = __reduce_add_sync(0xffffffffu, mine);
+  if (lane == 0) {
+    sc.red_min[warp] = kmin;
+    sc.red_max[warp] = kmax;
+    sc.warp_a[warp] = mine;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t a = __reduce_min_sync(0xffffffffu, lane < kRWarps ? sc.red_min[lane] : 0xffffffffu);
+    const uint32_t b = __reduce_max_sync(0xffffffffu, lane < kRWarps ? sc.red_max[lane] : 0u);
+    const int c = __reduce_add_sync(0xffffffffu, lane < kRWarps ? sc.warp_a[lane] : 0);
+    if (lane == 0) {
+      sc.loc_min = a;
+      sc.loc_max = b;
+      sc.loc_cnt = c;
+    }
+  }
+  csync<CS>(cl);                                   // every CTA's range is published
+  if (threadIdx.x == 0) {
+    uint32_t a = 0xffffffffu, b = 0u;
+    int c = 0;
+    for (int r = 0; r < CS; ++r) {
+      const RegShared* o = at_rank<CS>(cl, &sc, r);
+      a = min(a, o->loc_min);
+      b = max(b, o->loc_max);
+      c += o->loc_cnt;
+    }
+    sc.bcast[0] = (int)a;
+    sc.bcast[1] = (int)b;
+    sc.bcast[2] = c;
+  }
+  __syncthreads();
+  kmin = (uint32_t)sc.bcast[0];
+  kmax = (uint32_t)sc.bcast[1];
+  const int n_valid = sc.bcast[2];
+  __syncthreads();
+  for (int pass = 0; pass < 2; ++pass) {
+    const int k = pass == 0 ? K : Cout;
+    if (pass == 1 && cand_out == nullptr) break;
+    int32_t* out = pass == 0 ? topk_out + row * (size_t)K : cand_out + row * (size_t)Cout;
+    uint32_t T = 0u;
+    int need_eq = 0;
+    if (n_valid > k)
+      reg_threshold<KPT, CS>(cl, key, base, kmin, kmax, k, pass > 0, T, need_eq, sc);
+    reg_emit<KPT, CS>(cl, rank, key, base, T, need_eq, k, n_valid, crow, out, sc);
+  }
+  // no CTA leaves while the cluster may still read its shared memory
+  csync<CS>(cl);
+}
+
+template <int KPT, int CS>
+cudaError_t launch_topk_reg(const float* scores, int ld, const int32_t* nvalid,
+                            const int32_t* cand, int rows, int K, int32_t* topk_idx, int Cout,
+                            int32_t* cand_out, int* err, cudaStream_t stream) {
+  const dim3 grid((unsigned)(rows * CS)), cluster((unsigned)CS, 1, 1);
+  if (cand != nullptr)
+    return launch_pdl(topk_reg_kernel<KPT, CS, true>, grid, dim3(kRThreads), 0, stream, cluster,
+                      scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
+  return launch_pdl(topk_reg_kernel<KPT, CS, false>, grid, dim3(kRThreads), 0, stream, cluster,
+                    scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
+}
+
+template <int CS>
+cudaError_t launch_topk_reg_cs(const float* scores, int ld, const int32_t* nvalid,
+                               const int32_t* cand, int rows, int K, int32_t* topk_idx, int Cout,
+                               int32_t* cand_out, int* err, cudaStream_t stream) {
+  const int per = ceil_div(ceil_div(max(ld, 1), CS), kRThreads);
+  if (per <= 4)
+    return launch_topk_reg<4, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+  if (per <= 16)
+    return launch_topk_reg<16, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+  return launch_topk_reg<64, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+}
+
 }  // namespace
 
 int topk_sm_count() {
@@ -727,6 +1199,22 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
                         int rows, int K, int32_t* topk_idx, int Cout, int32_t* cand_out,
                         int* err, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
+  // Register variant: a cluster of CS CTAs per row (as many as keep rows x CS
+  // within the SMs), each holding at most 64 keys per thread in registers
+  {
+    const int sms = topk_sm_count();
+    int rcs = 1;
+    while (rcs < 8 && rows * rcs * 2 <= sms) rcs *= 2;
+    if (ld <= rcs * kRThreads * 64) {
+      if (rcs == 8)
+        return launch_topk_reg_cs<8>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+      if (rcs == 4)
+        return launch_topk_reg_cs<4>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+      if (rcs == 2)
+        return launch_topk_reg_cs<2>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+      return launch_topk_reg_cs<1>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+    }
+  }
   // Few rows: a cluster of cs CTAs per row (cs = 2, 4 or 8, as many as keep
   // rows x cs within one wave), each staging a slice of the row.
   const int sms = topk_sm_count();
