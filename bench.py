@@ -141,7 +141,8 @@ def profiled_traffic(kernel: str, workload: str, units: float):
 
 
 _NCU_SCALE = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "nsecond": 1e-3,
-              "usecond": 1.0, "msecond": 1e3, "second": 1e6}
+              "usecond": 1.0, "msecond": 1e3, "second": 1e6, "ns": 1e-3, "us": 1.0,
+              "ms": 1e3, "s": 1e6, "KB": 1e3, "MB": 1e6, "GB": 1e9, "B": 1.0}
 
 
 def record_ncu(csv_path: str, kernel: str, workload: str, command: str, units=None,

@@ -28,13 +28,13 @@
 // its part of the row sum live in registers. The maximum is lazy: P = 2^(s - m)
 // with m raised (and O and the row sum rescaled) only when a tile holds a logit
 // more than 8 above it, so P stays below 2^8 in fp16 and rescaling is rare.
-// Values are dequantised with integer ops (E2M1 magnitudes from a byte table,
-// E4M3 scales shifted into fp16 fields); they carry an exact factor 2^-8 that
-// the softmax scale and the epilogue undo. A producer dequantises a tile into
+// Values are dequantised exactly into fp16 by the hardware E2M1 and E4M3
+// conversions and one fp16 product per value. A producer dequantises a tile into
 // registers BEFORE waiting for its ring slot, so after the slot frees only the
 // shared-memory stores stand between P(t-3) V(t-3) and S(t).
-// Roles: warps 0-7 gather and dequantise; warp 8 owns tensor memory and issues
-// the MMAs; warps 9-12 stage Q into tensor memory and run the softmax. At the
+// Roles: warps 0-7 gather and dequantise, and stage Q into tensor memory after
+// the first tile; warp 8 owns tensor memory and issues the MMAs; warps 9-12 run
+// the softmax. At the
 // end every warp that can reach a quadrant's O lanes (its softmax warp and two
 // producer warps) writes that quadrant's output, partial or final. Every
 // mbarrier wait is bounded.
@@ -192,46 +192,75 @@ __device__ __forceinline__ uint32_t pack_bf162(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
+// Read-only global loads that the compiler keeps in program order among the
+// other volatile asm (shared-memory stores, barrier waits), so that a gather
+// issued a tile ahead is not sunk to its use.
+__device__ __forceinline__ uint2 ldg_v2(const void* ptr) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(ptr));
+  return r;
+}
+__device__ __forceinline__ uint4 ldg_v4(const void* ptr) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr));
+  return r;
+}
+__device__ __forceinline__ uint32_t ldg_u8(const void* ptr) {
+  uint32_t r;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(r) : "l"(ptr));
+  return r;
+}
+
+// Hardware conversions of packed FP4/FP8 pairs to f16x2 (the first, lower
+// nibble or byte into the lower half).
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t codes, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
+}
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t bytes, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 h0, h1;\n\t"
+      "mov.b32 {h0, h1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, h0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h1;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(bytes));
+}
+
 // 8 E2M1 codes (one 32-bit word, low nibble first) times their 8 E4M3 scales
-// (two words) -> one 16-byte chunk of fp16 values, times 2^-8. Integer ops only:
-//  - E2M1 magnitude m -> high byte of fp16(m) from an 8-entry byte table
-//    (0, 0.5, 1, 1.5, 2, 3, 4, 6 -> 00 38 3C 3E 40 42 44 46), sign spliced in;
-//  - a non-negative E4M3 byte shifted left by 7 is the fp16 of its value * 2^-8
-//    (exponent bias 7 -> 15, mantissa 3 -> 10 bits; subnormals line up too);
-//  - the fp16 product is exact (<= 6 significant bits, >= 2^-18).
+// (two words) -> one 16-byte chunk of fp16 values. The product is exact in
+// fp16: at most 6 significant bits, between 0.5 * 2^-9 and 6 * 448 = 2688.
 __device__ __forceinline__ uint4 dq8(uint32_t codes, uint32_t s_lo, uint32_t s_hi) {
-  const uint32_t mag = codes & 0x77777777u;
-  const uint32_t m_lo = __byte_perm(0x3E3C3800u, 0x46444240u, mag);         // codes 0-3
-  const uint32_t m_hi = __byte_perm(0x3E3C3800u, 0x46444240u, mag >> 16);   // codes 4-7
-  const uint32_t t = codes << 4;    // sign of each even code -> bit 7 of its byte
+  uint32_t v[4], sc[4];
+  e2m1x8_to_f16(codes, v);
+  e4m3x4_to_f16(s_lo, sc[0], sc[1]);
+  e4m3x4_to_f16(s_hi, sc[2], sc[3]);
   uint32_t h[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t mg = __byte_perm(j < 2 ? m_lo : m_hi, 0u, (j & 1) ? 0x3424u : 0x1404u);
-    const uint32_t sg = __byte_perm(t, codes, (uint32_t)((4 + j) * 0x1100 + j * 0x0011));
-    const uint32_t v = (mg & 0x7fff7fffu) | (sg & 0x80008000u);
-    const uint32_t sc = __byte_perm(j < 2 ? s_lo : s_hi, 0u, (j & 1) ? 0x4342u : 0x4140u) << 7;
-    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&v),
-                              *reinterpret_cast<const __half2*>(&sc));
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&v[j]),
+                              *reinterpret_cast<const __half2*>(&sc[j]));
     h[j] = *reinterpret_cast<const uint32_t*>(&r);
   }
   return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
 // 8 E4M3 bytes (two words, the first byte lowest) -> one 16-byte chunk of
-// fp16 values, times 2^-8 like the FP4 chunks: byte b becomes
-// ((b & 0x7f) << 7) | ((b & 0x80) << 8). *nan gets a nonzero bit for each
-// E4M3 NaN (0x7f, 0xff), whose fp16 pattern 0x3f80 no finite E4M3 value has.
+// fp16 values (exact: E4M3 is a subset of fp16). *nan gets a nonzero bit for
+// each E4M3 NaN byte (0x7f, 0xff).
 __device__ __forceinline__ uint4 e4m3x8(uint32_t a, uint32_t b, uint32_t* nan) {
-  uint32_t h[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    // halfwords (byte << 8) of bytes 2 (j & 1) and 2 (j & 1) + 1 of the word
-    const uint32_t x = __byte_perm(j < 2 ? a : b, 0u, (j & 1) ? 0x3424u : 0x1404u);
-    h[j] = (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
-    *nan |= __vcmpeq2(h[j] & 0x7fff7fffu, 0x3f803f80u);
-  }
-  return make_uint4(h[0], h[1], h[2], h[3]);
+  uint4 r;
+  e4m3x4_to_f16(a, r.x, r.y);
+  e4m3x4_to_f16(b, r.z, r.w);
+  *nan |= __vcmpeq4(a & 0x7f7f7f7fu, 0x7f7f7f7fu) | __vcmpeq4(b & 0x7f7f7f7fu, 0x7f7f7f7fu);
+  return r;
 }
 
 struct AttnParams {
@@ -414,23 +443,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         r[k].win = id <= -2;
         if (id <= -2) {
           const uint8_t* wr = swa_b + (size_t)(-2 - id) * kD + 16 * u;
-          r[k].s[0] = __ldg(reinterpret_cast<const uint4*>(wr));
-          r[k].s[1] = __ldg(reinterpret_cast<const uint4*>(wr + 256));
+          r[k].s[0] = ldg_v4(wr);
+          r[k].s[1] = ldg_v4(wr + 256);
         } else if (id >= 0) {
           const uint8_t* pr = pk_b + (size_t)id * kRowBytes + 8 * u;
-          r[k].c[0] = __ldg(reinterpret_cast<const uint2*>(pr));
-          r[k].c[1] = __ldg(reinterpret_cast<const uint2*>(pr + 128));
+          r[k].c[0] = ldg_v2(pr);
+          r[k].c[1] = ldg_v2(pr + 128);
           if (kG16) {
             // dims 16u .. 16u+15 are group u, dims 256+16u .. group 16+u: one
             // scale byte each, repeated for the eight dims of a dequantised chunk
             const uint8_t* sr = pk_b + (size_t)id * kRowBytes + kD / 2 + u;
-            const uint32_t s0 = 0x01010101u * __ldg(sr), s1 = 0x01010101u * __ldg(sr + 16);
+            const uint32_t s0 = 0x01010101u * ldg_u8(sr), s1 = 0x01010101u * ldg_u8(sr + 16);
             r[k].s[0] = make_uint4(s0, s0, s0, s0);
             r[k].s[1] = make_uint4(s1, s1, s1, s1);
           } else {
             const uint8_t* sr = sc_b + (size_t)(id / kBlockEntries) * kD + 16 * u;
-            r[k].s[0] = __ldg(reinterpret_cast<const uint4*>(sr));
-            r[k].s[1] = __ldg(reinterpret_cast<const uint4*>(sr + 256));
+            r[k].s[0] = ldg_v4(sr);
+            r[k].s[1] = ldg_v4(sr + 256);
           }
         } else {
           r[k].c[0] = r[k].c[1] = make_uint2(0, 0);
@@ -476,48 +505,65 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     };
     // ---- Q into tensor memory (lanes 0-15, columns 192 + d/2). The block's
     // query rows arrive by one bulk copy into V slot 2. Producer warps w and
-    // w + 4 convert quadrant w % 4's 16 rows in place, 8 rows each, a row at a
-    // time with all 32 lanes: bf16 -> fp16 scaled per head by a power of two (so
-    // every bf16 bit survives), 16-byte chunk c of row hh stored at chunk
-    // c ^ (hh & 7). Then thread (h, ch) of warp w moves dims 256 ch + 128 (w / 4)
-    // .. + 127 of row h into tensor memory. This overlaps the first gathers.
+    // w + 4 convert quadrant w % 4's 16 rows in place, 8 rows each, two rows
+    // at a time with all 32 lanes: bf16 -> fp16 scaled per head by a power of
+    // two (so every bf16 bit survives), 16-byte chunk c of row hh stored at chunk
+    // c ^ (hh & 7). A row's largest magnitude is taken on the bf16 bit patterns
+    // (non-negative floats order like their bits) with one warp reduction. Then
+    // thread (h, ch) of warp w moves dims 256 ch + 128 (w / 4) .. + 127 of row h
+    // into tensor memory. This runs after the first tile is published and
+    // overlaps the second tile's loads.
     auto stage_q = [&]() {
       const uint32_t qsm = vs_s + 2 * kVTile;
       bool ok = mbar_wait_warp(&sm.bar.q_ld, 0, abort_flag);
       if (ok) {
+        constexpr int kQRows = 2;
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-          const int hh = quad * 16 + (warp >> 2) * 8 + i;
-          if (hh >= nh) break;                                 // warp-uniform
-          const uint32_t qr = qsm + hh * 1024;
-          const uint4 a = lds128(qr + 16 * lane);
-          const uint4 c = lds128(qr + 512 + 16 * lane);
-          const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-          float amax = 0.0f;
+        for (int i0 = 0; i0 < 8; i0 += kQRows) {
+          uint4 a[kQRows], c[kQRows];
+          uint32_t amax[kQRows];
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
-                                     fabsf(__uint_as_float(w[k] & 0xffff0000u))));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-          // amax < 2^ex with ex from the exponent field; scaling by 2^e, e = 15 - ex,
-          // keeps every magnitude below 2^15 and is exact (clamped to |e| <= 100)
-          int ex2 = 0;
-          if (amax > 0.0f && isfinite(amax)) {
-            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-            ex2 = min(100, max(-100, 15 - ex));
+          for (int r = 0; r < kQRows; ++r) {
+            const int hh = quad * 16 + (warp >> 2) * 8 + i0 + r;
+            a[r] = c[r] = make_uint4(0, 0, 0, 0);
+            if (hh < nh) {                                   // warp-uniform
+              a[r] = lds128(qsm + hh * 1024 + 16 * lane);
+              c[r] = lds128(qsm + hh * 1024 + 512 + 16 * lane);
+            }
+            // |x| of 16 bf16 values as 16-bit integers, maximum by pairs
+            const uint32_t m = __vmaxu2(
+                __vmaxu2(__vmaxu2(a[r].x & 0x7fff7fffu, a[r].y & 0x7fff7fffu),
+                         __vmaxu2(a[r].z & 0x7fff7fffu, a[r].w & 0x7fff7fffu)),
+                __vmaxu2(__vmaxu2(c[r].x & 0x7fff7fffu, c[r].y & 0x7fff7fffu),
+                         __vmaxu2(c[r].z & 0x7fff7fffu, c[r].w & 0x7fff7fffu)));
+            amax[r] = __reduce_max_sync(0xffffffffu, max(m & 0xffffu, m >> 16));
           }
-          const float up = __uint_as_float((uint32_t)(127 + ex2) << 23);
-          uint32_t f[8];
+          __syncwarp();                                      // the rows are read before they are rewritten
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            f[k] = pack_half2(__uint_as_float(w[k] << 16) * up,
-                              __uint_as_float(w[k] & 0xffff0000u) * up);
-          __syncwarp();                                        // the row is read before it is rewritten
-          sts128(qr + ((lane ^ (hh & 7)) << 4), make_uint4(f[0], f[1], f[2], f[3]));
-          sts128(qr + (((32 + lane) ^ (hh & 7)) << 4), make_uint4(f[4], f[5], f[6], f[7]));
-          if (lane == 0) sm.qdown[hh] = __uint_as_float((uint32_t)(127 - ex2) << 23);
+          for (int r = 0; r < kQRows; ++r) {
+            const int hh = quad * 16 + (warp >> 2) * 8 + i0 + r;
+            if (hh >= nh) continue;                          // warp-uniform
+            // amax < 2^ex with ex from the exponent field; scaling by 2^e, e = 15 - ex,
+            // keeps every magnitude below 2^15 and is exact (clamped to |e| <= 100)
+            int ex2 = 0;
+            const uint32_t eb = (amax[r] >> 7) & 0xffu;      // bf16 exponent field
+            if (amax[r] != 0u && eb != 0xffu) {
+              // subnormal maxima (eb == 0) are below 2^-126: the clamp decides
+              const int ex = (int)eb - 126;
+              ex2 = min(100, max(-100, 15 - ex));
+            }
+            const float up = __uint_as_float((uint32_t)(127 + ex2) << 23);
+            const uint32_t w[8] = {a[r].x, a[r].y, a[r].z, a[r].w, c[r].x, c[r].y, c[r].z, c[r].w};
+            uint32_t f[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              f[k] = pack_half2(__uint_as_float(w[k] << 16) * up,
+                                __uint_as_float(w[k] & 0xffff0000u) * up);
+            const uint32_t qr = qsm + hh * 1024;
+            sts128(qr + ((lane ^ (hh & 7)) << 4), make_uint4(f[0], f[1], f[2], f[3]));
+            sts128(qr + (((32 + lane) ^ (hh & 7)) << 4), make_uint4(f[4], f[5], f[6], f[7]));
+            if (lane == 0) sm.qdown[hh] = __uint_as_float((uint32_t)(127 - ex2) << 23);
+          }
         }
       }
       __syncwarp();
@@ -568,7 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     Raw ra[2], rb[2];
     load_half(id_cur, ra, 0);
     load_half(id_cur, rb, 1);
-    stage_q();
+    // the query block is staged after the first tile (slot 0) is published, so
+    // its conversion overlaps the loads of the second; every split has a tile
+    if (nt == 0) stage_q();
     for (int t = 0; t < nt; ++t) {
       const int buf = t % kRing;
       uint4 dq[2][4];
@@ -588,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.v_full[buf]);
+      if (t == 0) stage_q();
       const int id_far_checked = check_index(id_far, t + 3);
       prefetch_rows(id_far_checked);
       id_far = fetch_index(t + 4);
@@ -642,12 +691,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         // buffer, are free once this has completed
         mma_commit(&sm.bar.v_free[buf]);
       };
-      for (int t = 0; ok && t < min(nt, kRing - 1); ++t) ok = issue_s(t);
+      if (ok && nt > 0) ok = issue_s(0);
       // Then whichever is ready first: P(t) V(t) once the softmax published P(t),
       // or S(t') (t' <= t + 2: its S and P buffers were released by the issue of
       // P(t'-3) V(t'-3), which completes before S(t')) once the producers
       // published its tile. Polling is bounded like mbar_wait.
-      int next_pv = 0, next_s = min(nt, kRing - 1);
+      int next_pv = 0, next_s = min(nt, 1);
       const uint64_t t0 = global_ns();
       uint32_t spins = 0;
       while (ok && next_pv < nt) {
@@ -679,8 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     const int h = quad * 16 + hl;                    // head of this thread within the block
     // the producers stage Q (and the per-head scales) first
     bool ok = mbar_wait_warp(&sm.bar.q_full, 0, abort_flag);
-    // x 2^8: the dequantised keys/values carry a factor 2^-8
-    const float hs = (ok && h < nh) ? p.softmax_scale * kLog2e * sm.qdown[h] * 256.0f : 0.0f;
+    const float hs = (ok && h < nh) ? p.softmax_scale * kLog2e * sm.qdown[h] : 0.0f;
     for (int t = 0; ok && t < nt; ++t) {
       const int buf = t % kRing;
       const uint32_t ph = (t / kRing) & 1;
@@ -772,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   // Every warp that reaches a quadrant's O lanes waits for the last P V, then
   // handles its chunks of the quadrant's 16 heads: the final output (one
   // split), the partial staged for the in-cluster merge, or the partial in the
-  // workspace. x 2^8 undoes the 2^-8 carried by the dequantised values.
+  // workspace.
   const bool writer = warp != kMmaWarp;
   bool have_o = false;
   if (writer) have_o = mbar_wait_warp(&sm.bar.o_full, 0, abort_flag);
@@ -801,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       if (h >= nh) continue;
       const int d0 = 256 * ch + 32 * c;           // this thread's dims d0 .. d0 + 31
       if (ns == 1) {
-        const float f = l_tot > 0.0f ? 256.0f / l_tot : 0.0f;
+        const float f = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
         uint4* dst = reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + h) * kD + d0);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -812,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       } else if (p.cluster_merge) {
         // normalised by this split's row sum (a convex combination of values,
         // |o| <= 2688, so fp16 holds it); nothing selected gives zeros
-        const float f = l_tot > 0.0f ? 256.0f / l_tot : 0.0f;
+        const float f = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int cl = d0 / 8 + k;                  // logical 16-byte chunk of the row
@@ -825,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       } else {
         // unnormalised, with the split's (max, sum), for the combine kernel;
         // a split with nothing selected contributes zeros
-        const float f = l_tot > 0.0f ? 256.0f : 0.0f;
+        const float f = l_tot > 0.0f ? 1.0f : 0.0f;
         float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * kHB + h) * kD + d0);
 #pragma unroll
         for (int k = 0; k < 8; ++k)

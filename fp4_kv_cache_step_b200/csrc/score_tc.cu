@@ -74,6 +74,10 @@ __device__ __forceinline__ void issue_tile(uint32_t d0, uint64_t ad, uint64_t bd
                bd + (uint64_t)((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
 }
 
+// kDecode: one query per group with 64 indexer heads (the weights stay in
+// registers); otherwise the general epilogue, so that each path gets the
+// registers it needs.
+template <bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap qmap, const TcParams p) {
@@ -249,7 +253,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       const int acc = k % p.nacc;
       const int b = g / p.groups_per_b;
       const int t0 = (g % p.groups_per_b) * p.nq;
-      if (p.nq == 1 && p.Hi == 64 && g != wg_group) {
+      if (kDecode && g != wg_group) {
         // load this query's weights and length once per group, before the wait
         const size_t row = (size_t)b * p.Tq + t0;
         const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * 64);
@@ -268,7 +272,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       tc_fence_after();
       const int j = (tile - tile_pre[g]) * (kTileM * p.sub) + m;
       const uint32_t acc_addr = tmem_base + lane_addr + (uint32_t)(acc * n_mma * p.sub);
-      if (p.nq == 1 && p.Hi == 64) {
+      if (kDecode) {
         float* dst = p.scores + ((size_t)b * p.Tq + t0) * p.N;
         for (int sb = 0; sb < p.sub; ++sb) {
           float v[64];
@@ -288,25 +292,48 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         continue;
       }
-      for (int qi = 0; qi < p.nq; ++qi) {
-        const int t = t0 + qi;
-        if (t >= p.Tq) break;                   // warp-uniform
-        const size_t row = (size_t)b * p.Tq + t;
-        const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * p.Hi);
-        float s = 0.0f;
-        for (int h0 = 0; h0 < p.Hi; h0 += 64) {
-          float v[64];
-          tmem_ld_64(acc_addr + (uint32_t)(qi * p.Hi + h0), v);
+      // the nq x Hi columns in pairs of 64-column chunks (one TMEM wait per
+      // pair); each chunk's 64 head terms go to 8 independent partial sums
+      // (integer-valued terms add exactly in any order)
+      const int nchunk = p.nq * (p.Hi / 64);
+      float part = 0.0f;                        // Hi = 128: the first half's sum
+      for (int c0 = 0; c0 < nchunk; c0 += 2) {
+        float va[64], vb[64];
+        const bool two = c0 + 1 < nchunk;
+        tmem_ld_64x2(acc_addr + (uint32_t)(c0 * 64), acc_addr + (uint32_t)((two ? c0 + 1 : c0) * 64),
+                     va, vb);
 #pragma unroll
-          for (int i = 0; i < 64; i += 4) {
-            const float4 wv = __ldg(w4 + (h0 + i) / 4);
-            s = fmaf(wv.x, fmaxf(v[i], 0.0f), s);
-            s = fmaf(wv.y, fmaxf(v[i + 1], 0.0f), s);
-            s = fmaf(wv.z, fmaxf(v[i + 2], 0.0f), s);
-            s = fmaf(wv.w, fmaxf(v[i + 3], 0.0f), s);
+        for (int half = 0; half < 2; ++half) {
+          const int c = c0 + half;
+          if (c >= nchunk) break;
+          const float* v = half ? vb : va;
+          const int qi = c / (p.Hi / 64), h0 = (c % (p.Hi / 64)) * 64;
+          const int t = t0 + qi;
+          if (t >= p.Tq) break;                 // warp-uniform
+          const size_t row = (size_t)b * p.Tq + t;
+          const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * p.Hi + h0);
+          float acc8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int i = 0; i < 64; i += 8) {
+            const float4 wa = __ldg(w4 + i / 4), wb = __ldg(w4 + i / 4 + 1);
+            acc8[0] = fmaf(wa.x, fmaxf(v[i], 0.0f), acc8[0]);
+            acc8[1] = fmaf(wa.y, fmaxf(v[i + 1], 0.0f), acc8[1]);
+            acc8[2] = fmaf(wa.z, fmaxf(v[i + 2], 0.0f), acc8[2]);
+            acc8[3] = fmaf(wa.w, fmaxf(v[i + 3], 0.0f), acc8[3]);
+            acc8[4] = fmaf(wb.x, fmaxf(v[i + 4], 0.0f), acc8[4]);
+            acc8[5] = fmaf(wb.y, fmaxf(v[i + 5], 0.0f), acc8[5]);
+            acc8[6] = fmaf(wb.z, fmaxf(v[i + 6], 0.0f), acc8[6]);
+            acc8[7] = fmaf(wb.w, fmaxf(v[i + 7], 0.0f), acc8[7]);
+          }
+          const float s = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
+                          ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+          float* dst = p.scores + row * p.N + j;
+          if (j < min(p.nvalid[row], p.N)) {
+            if (p.Hi == 64) *dst = s;
+            else if (h0 == 0) part = s;         // Hi = 128: two chunks per query
+            else *dst = part + s;
           }
         }
-        if (j < min(p.nvalid[row], p.N)) p.scores[row * p.N + j] = s;
       }
       tc_fence_before();
       __syncwarp();
@@ -407,14 +434,16 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
     return cudaErrorInvalidValue;
 
   const size_t smem = fixed + (size_t)p.stages * tile_bytes;
-  cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool dec = p.nq == 1 && Hi == 64;
+  void (*kernel)(CUtensorMap, CUtensorMap, TcParams) =
+      dec ? index_score_tc_kernel<true> : index_score_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   // upper bound on the tile count; CTAs beyond the real count get empty ranges
   const long long max_tiles = (long long)p.G * ((N + kTileM * p.sub - 1) / (kTileM * p.sub));
   const int grid = (int)std::min<long long>(sm_count(), std::max<long long>(1, max_tiles));
-  return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kThreads), smem, stream, dim3(1),
-                    kmap, qmap, p);
+  return launch_pdl(kernel, dim3(grid), dim3(kThreads), smem, stream, dim3(1), kmap, qmap, p);
 }
 
 }  // namespace csa2

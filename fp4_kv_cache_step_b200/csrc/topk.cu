@@ -741,20 +741,24 @@ constexpr int kRWarps = kRThreads / 32;
 constexpr int kRBins = 4096;
 constexpr int kRBinsPerThread = kRBins / kRThreads;
 constexpr int kRCandCap = 1024;
+constexpr int kRGroups = 64;                      // groups of 64 bins
 
 struct __align__(16) RegShared {
-  int bins[kRBins];                 // this CTA's histogram (read by the cluster)
+  int bins[kRBins];                 // this CTA's histogram (fine bins read by the cluster)
   uint32_t cand_key[kRCandCap];     // this CTA's keys in the threshold bin (read by the cluster)
   int cand_pos[kRCandCap];
   uint32_t all_key[kRCandCap];      // the whole row's threshold bin
   int all_pos[kRCandCap];
+  // written by every CTA of the cluster into every CTA (slot = the writer's
+  // rank), so that after a cluster barrier each CTA reads them locally
+  int coarse[8][kRGroups];          // per rank: its counts of 64 groups of 64 bins (descending)
+  uint32_t rng_min[8], rng_max[8];  // per rank: its key range and count of real keys
+  int rng_cnt[8];
+  uint32_t emit_from[2][8];         // per pass and rank: its (greater << 16 | equal) counts
   int warp_a[kRWarps], warp_b[kRWarps];
   uint32_t red_min[kRWarps], red_max[kRWarps];
-  int bcast[4];
+  int bcast[8];
   int ncand;
-  uint32_t loc_min, loc_max;        // this CTA's key range and count (read by the cluster)
-  int loc_cnt;
-  uint32_t loc_emit;                // this CTA's (greater << 16 | equal) counts (read by the cluster)
 };
 
 template <int CS>
@@ -773,43 +777,32 @@ __device__ __forceinline__ int reg_pos(int base, int j, int q) {
   return base + (int)(threadIdx.x >> 5) * 32 * KPT + 128 * j + 4 * (int)(threadIdx.x & 31) + q;
 }
 
-// Exclusive prefix sum of v over the block (thread order).
-__device__ __forceinline__ int reg_block_scan(int v, int& total, RegShared& sc) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+// Inclusive prefix sum over the 32 lanes of a warp.
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
+    const int u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
   }
-  if (lane == 31) sc.warp_a[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int w = lane < kRWarps ? sc.warp_a[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
-    }
-    if (lane < kRWarps) sc.warp_b[lane] = wi - w;
-    if (lane == 31) sc.bcast[3] = wi;
-  }
-  __syncthreads();
-  const int res = sc.warp_b[warp] + incl - v;
-  total = sc.bcast[3];
-  __syncthreads();
-  return res;
+  return v;
 }
 
 // (T, need_eq) of the k-th largest real key of the row (1 <= k <= its real
 // keys): T is the key, need_eq how many keys equal to T the selection takes.
 // `reads_pending`: the cluster may still read this CTA's histogram or
 // candidates from an earlier call.
+// Per digit: each CTA counts its keys into 4096 bins over the current range
+// and writes its 64 group counts (64 bins each, descending) into every CTA;
+// after one cluster barrier warp 0 of each CTA finds, locally, the group that
+// holds the k-th key, then reads that group's 64 bins from every CTA and finds
+// the bin.
 template <int KPT, int CS>
 __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT], int base,
                               uint32_t kmin, uint32_t kmax, int k, bool reads_pending,
                               uint32_t& T, int& need_eq, RegShared& sc) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = CS > 1 ? (int)cl.block_rank() : 0;
   uint32_t lo = kmin;
   uint32_t width_m1 = kmax - kmin;                 // range [lo, lo + width_m1]
   const int bits = width_m1 == 0u ? 0 : 32 - __clz(width_m1);
@@ -817,7 +810,8 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
   int krem = k;
   bool first = true;
   for (;;) {
-    if (CS > 1 && (reads_pending || !first)) cl.sync();   // nobody still reads our histogram
+    // nobody still reads our histogram or our group counts
+    if (CS > 1 && (reads_pending || !first)) cl.sync();
     for (int i = threadIdx.x; i < kRBins; i += kRThreads) sc.bins[i] = 0;
     if (threadIdx.x == 0) sc.ncand = 0;
     __syncthreads();
@@ -834,37 +828,64 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
       }
     }
     first = false;
-    csync<CS>(cl);                                 // the cluster's histograms are complete
-    // descending bins: thread t owns bins 4095 - 8t .. 4088 - 8t, summed over the cluster
-    const int b0 = kRBins - kRBinsPerThread * ((int)threadIdx.x + 1);
-    int loc[kRBinsPerThread] = {0, 0, 0, 0, 0, 0, 0, 0};
+    __syncthreads();
+    {
+      // thread t sums bins 4095 - 8t .. 4088 - 8t; 8 threads make group t / 8
+      const int b0 = kRBins - kRBinsPerThread * ((int)threadIdx.x + 1);
+      const int4 x = *reinterpret_cast<const int4*>(sc.bins + b0);
+      const int4 y = *reinterpret_cast<const int4*>(sc.bins + b0 + 4);
+      int s8 = x.x + x.y + x.z + x.w + y.x + y.y + y.z + y.w;
+      s8 += __shfl_xor_sync(0xffffffffu, s8, 1);
+      s8 += __shfl_xor_sync(0xffffffffu, s8, 2);
+      s8 += __shfl_xor_sync(0xffffffffu, s8, 4);
+      if ((lane & 7) == 0) {
+        const int g = (int)threadIdx.x >> 3;
 #pragma unroll
-    for (int r = 0; r < CS; ++r) {
-      const int4* src = reinterpret_cast<const int4*>(at_rank<CS>(cl, sc.bins, r) + b0);
-      const int4 x = src[0], y = src[1];
-      loc[0] += y.w;
-      loc[1] += y.z;
-      loc[2] += y.y;
-      loc[3] += y.x;
-      loc[4] += x.w;
-      loc[5] += x.z;
-      loc[6] += x.y;
-      loc[7] += x.x;
+        for (int r = 0; r < CS; ++r) at_rank<CS>(cl, &sc.coarse[rank][g], r)[0] = s8;
+      }
     }
-    int mine = 0;
+    csync<CS>(cl);                                 // every CTA's group counts are everywhere
+    if (warp == 0) {
+      // groups 2 lane and 2 lane + 1, summed over the cluster
+      int c0 = 0, c1 = 0;
 #pragma unroll
-    for (int j = 0; j < kRBinsPerThread; ++j) mine += loc[j];
-    int tot;
-    int above = reg_block_scan(mine, tot, sc);
-    if (above < krem && krem <= above + mine) {
+      for (int r = 0; r < CS; ++r) {
+        c0 += sc.coarse[r][2 * lane];
+        c1 += sc.coarse[r][2 * lane + 1];
+      }
+      const int incl = warp_incl_scan(c0 + c1);
+      const int before = incl - c0 - c1;
+      int g = -1, kg = 0;
+      if (before < krem && krem <= before + c0) {
+        g = 2 * lane;
+        kg = krem - before;
+      } else if (before + c0 < krem && krem <= incl) {
+        g = 2 * lane + 1;
+        kg = krem - before - c0;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, g >= 0);
+      const int src = hit ? __ffs(hit) - 1 : 0;      // exactly one lane holds the k-th key
+      g = max(0, __shfl_sync(0xffffffffu, g, src));
+      kg = __shfl_sync(0xffffffffu, kg, src);
+      // its 64 bins, descending: bin top - 2 lane and top - 2 lane - 1
+      const int top = kRBins - 1 - 64 * g;
+      int f0 = 0, f1 = 0;
 #pragma unroll
-      for (int j = 0; j < kRBinsPerThread; ++j) {
-        if (above < krem && krem <= above + loc[j]) {
-          sc.bcast[0] = kRBins - 1 - kRBinsPerThread * (int)threadIdx.x - j;
-          sc.bcast[1] = krem - above;
-          sc.bcast[2] = loc[j];
-        }
-        above += loc[j];
+      for (int r = 0; r < CS; ++r) {
+        const int* br = at_rank<CS>(cl, sc.bins, r);
+        f0 += br[top - 2 * lane];
+        f1 += br[top - 2 * lane - 1];
+      }
+      const int fi = warp_incl_scan(f0 + f1);
+      const int fb = fi - f0 - f1;
+      if (fb < kg && kg <= fb + f0) {
+        sc.bcast[0] = top - 2 * lane;
+        sc.bcast[1] = kg - fb;
+        sc.bcast[2] = f0;
+      } else if (fb + f0 < kg && kg <= fi) {
+        sc.bcast[0] = top - 2 * lane - 1;
+        sc.bcast[1] = kg - fb - f0;
+        sc.bcast[2] = f1;
       }
     }
     __syncthreads();
@@ -898,19 +919,22 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
       const uint32_t* ck = sc.cand_key;
       const int* cp = sc.cand_pos;
       if (CS > 1) {
-        int off = 0;
-        for (int r = 0; r < CS; ++r) {
-          RegShared* o = at_rank<CS>(cl, &sc, r);
-          const int nr = min(o->ncand, kRCandCap);
-          for (int u = threadIdx.x; u < nr; u += kRThreads) {
-            if (off + u < kRCandCap) {
-              sc.all_key[off + u] = o->cand_key[u];
-              sc.all_pos[off + u] = o->cand_pos[u];
-            }
-          }
-          off += nr;
+        // every CTA's count first (independent loads), then one pass over all
+        int nr[CS], off[CS + 1];
+#pragma unroll
+        for (int r = 0; r < CS; ++r) nr[r] = min(at_rank<CS>(cl, &sc, r)->ncand, kRCandCap);
+        off[0] = 0;
+#pragma unroll
+        for (int r = 0; r < CS; ++r) off[r + 1] = off[r] + nr[r];
+        c = min(off[CS], kRCandCap);
+        for (int u = threadIdx.x; u < c; u += kRThreads) {
+          int r = 0;
+#pragma unroll
+          for (int q = 1; q < CS; ++q) r += u >= off[q];
+          const RegShared* o = at_rank<CS>(cl, &sc, r);
+          sc.all_key[u] = o->cand_key[u - off[r]];
+          sc.all_pos[u] = o->cand_pos[u - off[r]];
         }
-        c = min(off, kRCandCap);
         ck = sc.all_key;
         cp = sc.all_pos;
         __syncthreads();
@@ -947,9 +971,9 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
 // Writes, in position order, every key above T and the first need_eq keys equal
 // to T (T = 0 selects every real key), then pads with -1 up to k.
 template <int KPT, int CS>
-__device__ void reg_emit(cg::cluster_group& cl, int rank, const uint32_t (&key)[KPT], int base,
-                         uint32_t T, int need_eq, int k, int n_valid, const int32_t* crow,
-                         int32_t* out, RegShared& sc) {
+__device__ void reg_emit(cg::cluster_group& cl, int rank, int pass, const uint32_t (&key)[KPT],
+                         int base, uint32_t T, int need_eq, int k, int n_valid,
+                         const int32_t* crow, int32_t* out, RegShared& sc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // (greater << 16 | equal) counts: a CTA's totals (at most 512 x 64) fit 16 bits each
   uint32_t c = 0;
@@ -967,13 +991,15 @@ __device__ void reg_emit(cg::cluster_group& cl, int rank, const uint32_t (&key)[
       if (lane >= o) incl += u;
     }
     if (lane < kRWarps) sc.warp_b[lane] = (int)(incl - v);
-    if (lane == 31) sc.loc_emit = incl;
+    // this CTA's totals (lane 31's inclusive sum) into every later CTA
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane < CS && lane > rank) at_rank<CS>(cl, &sc.emit_from[pass][rank], lane)[0] = total;
   }
   csync<CS>(cl);                                   // every CTA's counts are published
   // selected before this warp's first chunk row: the earlier CTAs' and warps'
   int gt_run = 0, eq_run = 0;
   for (int r = 0; r < rank; ++r) {
-    const uint32_t e = at_rank<CS>(cl, &sc, r)->loc_emit;
+    const uint32_t e = sc.emit_from[pass][r];
     gt_run += (int)(e >> 16);
     eq_run += (int)(e & 0xffffu);
   }
@@ -1023,6 +1049,9 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
                 int Cout, int32_t* __restrict__ cand_out, int* err) {
   static_assert(KPT % 4 == 0 && KPT <= 64, "chunks of four keys, at most 64 per thread");
   __shared__ RegShared sc;
+  // every CTA of the cluster must be running before any writes into another's
+  // shared memory: arrive now, wait just before the first such write
+  if (CS > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   pdl_wait_and_release();
   cg::cluster_group cl = cg::this_cluster();
   const int rank = CS > 1 ? (int)cl.block_rank() : 0;
@@ -1119,35 +1148,28 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
     sc.warp_a[warp] = mine;
   }
   __syncthreads();
+  if (CS > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");   // all threads
   if (warp == 0) {
     const uint32_t a = __reduce_min_sync(0xffffffffu, lane < kRWarps ? sc.red_min[lane] : 0xffffffffu);
     const uint32_t b = __reduce_max_sync(0xffffffffu, lane < kRWarps ? sc.red_max[lane] : 0u);
     const int c = __reduce_add_sync(0xffffffffu, lane < kRWarps ? sc.warp_a[lane] : 0);
-    if (lane == 0) {
-      sc.loc_min = a;
-      sc.loc_max = b;
-      sc.loc_cnt = c;
+    // this CTA's range and count into every CTA of the cluster
+    if (lane < CS) {
+      at_rank<CS>(cl, &sc.rng_min[rank], lane)[0] = a;
+      at_rank<CS>(cl, &sc.rng_max[rank], lane)[0] = b;
+      at_rank<CS>(cl, &sc.rng_cnt[rank], lane)[0] = c;
     }
   }
-  csync<CS>(cl);                                   // every CTA's range is published
-  if (threadIdx.x == 0) {
-    uint32_t a = 0xffffffffu, b = 0u;
-    int c = 0;
-    for (int r = 0; r < CS; ++r) {
-      const RegShared* o = at_rank<CS>(cl, &sc, r);
-      a = min(a, o->loc_min);
-      b = max(b, o->loc_max);
-      c += o->loc_cnt;
-    }
-    sc.bcast[0] = (int)a;
-    sc.bcast[1] = (int)b;
-    sc.bcast[2] = c;
+  csync<CS>(cl);                                   // every CTA's range is everywhere
+  kmin = 0xffffffffu;
+  kmax = 0u;
+  int n_valid = 0;
+#pragma unroll
+  for (int r = 0; r < CS; ++r) {
+    kmin = min(kmin, sc.rng_min[r]);
+    kmax = max(kmax, sc.rng_max[r]);
+    n_valid += sc.rng_cnt[r];
   }
-  __syncthreads();
-  kmin = (uint32_t)sc.bcast[0];
-  kmax = (uint32_t)sc.bcast[1];
-  const int n_valid = sc.bcast[2];
-  __syncthreads();
   for (int pass = 0; pass < 2; ++pass) {
     const int k = pass == 0 ? K : Cout;
     if (pass == 1 && cand_out == nullptr) break;
@@ -1156,10 +1178,11 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
     int need_eq = 0;
     if (n_valid > k)
       reg_threshold<KPT, CS>(cl, key, base, kmin, kmax, k, pass > 0, T, need_eq, sc);
-    reg_emit<KPT, CS>(cl, rank, key, base, T, need_eq, k, n_valid, crow, out, sc);
+    reg_emit<KPT, CS>(cl, rank, pass, key, base, T, need_eq, k, n_valid, crow, out, sc);
   }
-  // no CTA leaves while the cluster may still read its shared memory
-  csync<CS>(cl);
+  // Every access to another CTA's shared memory (the fine bins, the candidate
+  // lists, and the values written into every CTA) precedes the last cluster
+  // barrier in reg_emit, so a CTA may leave without waiting for the others.
 }
 
 template <int KPT, int CS>

@@ -75,8 +75,12 @@ def test_pack_saturates_and_flags_nonfinite():
 
 
 # ------------------------------------------------------------------ indexer
+# (3, 2, 1024, 64, 128), (1, 5, 2048, 64, 128) and (2, 3, 1024, 128, 128) take
+# the tensor-core scorer's multi-query path (groups of 4 and 2 queries, the
+# last group partial; 128 heads in two 64-column chunks per query)
 @pytest.mark.parametrize("B,Tq,N,Hi,Di", [(1, 1, 4096, 4, 64), (3, 2, 1000 // 64 * 64 + 64, 64, 128),
-                                          (2, 3, 640, 16, 32)])
+                                          (2, 3, 640, 16, 32), (1, 5, 2048, 64, 128),
+                                          (2, 3, 1024, 128, 128)])
 def test_index_score_exact(B, Tq, N, Hi, Di):
     rng = np.random.default_rng(N + Hi)
     qb = _e4m3(rng.integers(-4, 5, (B, Tq, Hi, Di)))
