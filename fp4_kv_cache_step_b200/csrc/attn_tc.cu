@@ -68,7 +68,7 @@ constexpr float kRescaleSlack = 8.0f;    // log2 units: P <= 2^8 before a rescal
 constexpr int kMaxClusterSplits = 8;
 
 struct __align__(8) Bars {
-  uint64_t q_ld, q_conv, q_full, q_free, o_full, recv;
+  uint64_t q_ld, q_conv, q_full, q_free, o_full;
   uint64_t v_full[kRing], v_free[kRing], s_full[kRing], p_full[kRing];
 };
 
@@ -89,14 +89,14 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 // stages its partial output of every head, normalised by its own row sum and
 // rounded to fp16, grouped by the split that merges the head ([owner r][head hh
 // of r's share][512], 1 KB rows whose 16-byte chunks are swizzled by hh), with
-// its (max, sum) pairs; bulk copies then move each group into its owner's
-// receive area ([source split r][hh][512]); the owner merges its heads.
+// its (max, sum) pairs; every thread then copies 16-byte pieces of each group
+// into its owner's receive area ([source split r][hh][512]) through
+// distributed shared memory; the owner merges its heads.
 constexpr uint32_t kMergeSendOff = 0;               // bytes into the V region
 constexpr uint32_t kMergeSendMlOff = 72 * 1024;
 constexpr uint32_t kMergeRecvOff = 76 * 1024;
 constexpr uint32_t kMergeRecvMlOff = 148 * 1024;
-constexpr uint32_t kMergeWtsOff = 152 * 1024;
-static_assert(kMergeWtsOff + 32 * kMaxClusterSplits * sizeof(float) <= (size_t)kRing * kVTile,
+static_assert(kMergeRecvMlOff + 4 * 1024 <= (size_t)kRing * kVTile,
               "merge staging fits in the V region");
 // heads each split of a cluster of ns merges, and the 16-byte-padded bytes of
 // their (max, sum) pairs
@@ -337,7 +337,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     mbar_init(&sm.bar.q_full, kProducerWarps);
     mbar_init(&sm.bar.q_free, kProducerWarps);
     mbar_init(&sm.bar.o_full, 1);
-    mbar_init(&sm.bar.recv, 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&sm.bar.v_full[i], kProducerWarps);
       mbar_init(&sm.bar.v_free[i], 1);
@@ -830,8 +829,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   const int ns = p.nsplit;
   const int share = merge_share(ns);                   // heads each split of a cluster merges
   const uint32_t mlb = merge_ml_bytes(ns);
-  if (p.cluster_merge && threadIdx.x == 0)
-    mbar_arrive_expect_tx(&sm.bar.recv, (uint32_t)(ns - 1) * ((uint32_t)share * 1024u + mlb));
   if (writer && have_o) {
     const int hl = lane & 15, ch = lane >> 4;
     const int h = quad * 16 + hl;
@@ -892,7 +889,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
         p.ws_ml[slot * kHB + h] = mlh;
       }
     }
-    if (p.cluster_merge) fence_async_smem();      // the staging is read by bulk copies
   }
   tc_fence_before();
   __syncthreads();
@@ -902,26 +898,33 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
   }
 
   if (p.cluster_merge) {
-    // Every split has staged its partials and left its V region idle. Split s
-    // sends its group for owner r into r's receive area, slot s, and merges the
-    // heads [s share, (s + 1) share) from its own group and the ones it received:
-    // out = sum_r w_r o_r with o_r the partial normalised by its row sum l_r,
-    // w_r = 2^(m_r - M) l_r / L, L = sum_r 2^(m_r - M) l_r, M = max_r m_r.
+    // Every split has staged its partials and, after the first cluster
+    // barrier, every V region is idle. Split s copies its group for owner r into
+    // r's receive area, slot s (all threads, 16 bytes at a time through
+    // distributed shared memory); after the second barrier each split merges
+    // the heads [s share, (s + 1) share) from its own group and the ones it
+    // received: out = sum_r w_r o_r with o_r the partial normalised by its row
+    // sum l_r, w_r = 2^(m_r - M) l_r / L, L = sum_r 2^(m_r - M) l_r,
+    // M = max_r m_r. No shared memory of another CTA is touched after the
+    // second barrier, so a split may leave as soon as its merge is written.
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();
-    if (threadIdx.x == 0) {
-      const uint32_t recv_bar = smem_u32(&sm.bar.recv);
+    {
+      const uint32_t blk = (uint32_t)share * 1024u;
       for (int r = 0; r < ns; ++r) {
         if (r == split) continue;
-        bulk_copy_to_peer(
-            cluster_addr(smem_u32(vs + kMergeRecvOff + (size_t)split * share * 1024), (uint32_t)r),
-            vs + kMergeSendOff + (size_t)r * share * 1024, (uint32_t)share * 1024u,
-            cluster_addr(recv_bar, (uint32_t)r));
-        bulk_copy_to_peer(cluster_addr(smem_u32(vs + kMergeRecvMlOff + split * mlb), (uint32_t)r),
-                          vs + kMergeSendMlOff + r * mlb, mlb, cluster_addr(recv_bar, (uint32_t)r));
+        const uint32_t src = vs_s + kMergeSendOff + (uint32_t)r * blk;
+        const uint32_t dst = cluster_addr(vs_s + kMergeRecvOff + (uint32_t)split * blk, (uint32_t)r);
+        for (uint32_t o = 16u * threadIdx.x; o < blk; o += 16u * kThreads)
+          st_cluster128(dst + o, lds128(src + o));
+        const uint32_t msrc = vs_s + kMergeSendMlOff + (uint32_t)r * mlb;
+        const uint32_t mdst = cluster_addr(vs_s + kMergeRecvMlOff + (uint32_t)split * mlb, (uint32_t)r);
+        for (uint32_t o = 16u * threadIdx.x; o < mlb; o += 16u * kThreads)
+          st_cluster128(mdst + o, lds128(msrc + o));
       }
     }
-    const bool got = mbar_wait_warp(&sm.bar.recv, 0, abort_flag);
+    cl.sync();
+    const bool got = !*abort_flag;
     const int hA = split * share, hB = min(nh, hA + share);
     const int nhm = max(0, hB - hA);
     auto part_row = [&](int r, int i) -> uint32_t {
@@ -932,57 +935,54 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       return r == split ? reinterpret_cast<const float2*>(vs + kMergeSendMlOff + split * mlb)[i]
                         : reinterpret_cast<const float2*>(vs + kMergeRecvMlOff + r * mlb)[i];
     };
-    float* wts = reinterpret_cast<float*>(vs + kMergeWtsOff);    // [own head][8 splits]
-    if (got) {
-      for (int i = threadIdx.x; i < nhm; i += kThreads) {
-        float M = -INFINITY;
-        for (int r = 0; r < ns; ++r) M = fmaxf(M, part_ml(r, i).x);
-        float w[kMaxClusterSplits];
-        float L = 0.0f;
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r) {
-          w[r] = 0.0f;
-          if (r < ns) {
-            const float2 ml = part_ml(r, i);
-            w[r] = (ml.x != -INFINITY && ml.y > 0.0f) ? exp2f(ml.x - M) * ml.y : 0.0f;
-            L += w[r];
-          }
-        }
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-#pragma unroll
-        for (int r = 0; r < kMaxClusterSplits; ++r) wts[i * kMaxClusterSplits + r] = w[r] * inv;
-        if (p.lse) p.lse[row * p.Hq + h0 + hA + i] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-    const int units = got ? nhm * (kD / 8) : 0;        // 16-byte chunks of 8 fp16
+    // one 16-byte chunk (8 dims) of one head per unit; every split's (max, sum)
+    // and chunk are loaded first, then the weights and the sum
+    const int units = got ? nhm * (kD / 8) : 0;
 #pragma unroll 1
     for (int uo = threadIdx.x; uo < units; uo += kThreads) {
-      const int i = uo / (kD / 8), cl = uo % (kD / 8);
-      const int off = (cl ^ (i & 7)) << 4;
-      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+      const int i = uo / (kD / 8), cl16 = uo % (kD / 8);
+      const int off = (cl16 ^ (i & 7)) << 4;
+      float2 ml[kMaxClusterSplits];
+      uint4 v[kMaxClusterSplits];
 #pragma unroll
       for (int r = 0; r < kMaxClusterSplits; ++r) {
         if (r < ns) {
-          const float wr = wts[i * kMaxClusterSplits + r];
-          if (wr != 0.0f) {
-            const uint4 v = lds128(part_row(r, i) + off);
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
-              acc[2 * k] = fmaf(wr, f2.x, acc[2 * k]);
-              acc[2 * k + 1] = fmaf(wr, f2.y, acc[2 * k + 1]);
-            }
-          }
+          ml[r] = part_ml(r, i);
+          v[r] = lds128(part_row(r, i) + off);
+        } else {
+          ml[r] = make_float2(-INFINITY, 0.0f);
+          v[r] = make_uint4(0, 0, 0, 0);
         }
       }
-      *reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 8 * cl) =
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kMaxClusterSplits; ++r) M = fmaxf(M, ml[r].x);
+      float w[kMaxClusterSplits];
+      float L = 0.0f;
+#pragma unroll
+      for (int r = 0; r < kMaxClusterSplits; ++r) {
+        w[r] = (ml[r].x != -INFINITY && ml[r].y > 0.0f) ? fast_exp2(ml[r].x - M) * ml[r].y : 0.0f;
+        L += w[r];
+      }
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+      float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int r = 0; r < kMaxClusterSplits; ++r) {
+        const float wr = w[r] * inv;
+        const uint32_t vw[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
+          acc[2 * k] = fmaf(wr, f2.x, acc[2 * k]);
+          acc[2 * k + 1] = fmaf(wr, f2.y, acc[2 * k + 1]);
+        }
+      }
+      *reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 8 * cl16) =
           make_uint4(pack_bf162(acc[0], acc[1]), pack_bf162(acc[2], acc[3]),
                      pack_bf162(acc[4], acc[5]), pack_bf162(acc[6], acc[7]));
+      if (cl16 == 0 && p.lse)
+        p.lse[row * p.Hq + h0 + hA + i] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
-    // no split leaves while a bulk copy may still read its staging
-    cl.sync();
   }
   if (threadIdx.x == 0 && *abort_flag) record_error(p.err, CSA2_ERR_TIMEOUT);
 }

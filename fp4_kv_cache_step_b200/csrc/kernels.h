@@ -132,6 +132,12 @@ struct SwaWindow {
   int Tw, W;
 };
 
+// The blockwise pool of blocks of 8 in one launch of the register top-K (true
+// when it applied; *e holds the launch status).
+bool launch_block_pool_reg(const float* scores, int ld, const int32_t* nvalid, int rows,
+                           int block, int nblocks, int32_t* cand, int* err, cudaStream_t stream,
+                           cudaError_t* e);
+
 // Sparse attention; see csa2_sparse_attn. With kv_scale NULL, kv_packed holds
 // the 16-channel layout (csa2_sparse_attn_g16): per entry D/2 code bytes then
 // D/16 E4M3 scale bytes. With swa non-null the window branch joins the same

@@ -12,7 +12,9 @@
 //   launch_topk        the best nblocks blocks, ascending block ids
 //   block_expand_kernel block ids -> their valid positions, ascending, -1 padded
 // All three are small next to the scan that produced the scores (4 bytes read
-// per valid position, from L2 right after the scorer wrote them).
+// per valid position, from L2 right after the scorer wrote them). For blocks
+// of 8 the register top-K does all three in one launch (block mode: keys are
+// block maxima, the kept blocks written as their positions).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,6 +95,11 @@ cudaError_t launch_block_pool(const float* scores, int ld, const int32_t* nvalid
   const int nbmax = (int)(((size_t)ld + block - 1) / block);
   if (nbmax == 0)   // no position at all: an empty pool (all bytes 0xff = -1)
     return cudaMemsetAsync(cand, 0xff, (size_t)rows * nblocks * block * sizeof(int32_t), stream);
+  // blocks of 8 (the pages' size) in one launch: the register top-K keys each
+  // block by its maximum and writes the kept blocks' positions itself
+  cudaError_t er = cudaSuccess;
+  if (launch_block_pool_reg(scores, ld, nvalid, rows, block, nblocks, cand, err, stream, &er))
+    return er;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   float* bscores = reinterpret_cast<float*>(ws);
   int32_t* nvb = reinterpret_cast<int32_t*>(ws + align_up((size_t)rows * nbmax * sizeof(float)));

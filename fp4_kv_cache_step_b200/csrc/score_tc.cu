@@ -36,6 +36,7 @@ using namespace sm100;
 
 constexpr int kTileM = 128;
 constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;                // warps 2-9
 constexpr int kMaxGroups = 8192;
 constexpr size_t kSmemLimit = 227 * 1024;   // opt-in dynamic shared memory per CTA
 
@@ -90,7 +91,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   const int q_bytes = n_mma * p.Di;
   uint8_t* kbuf = base;
   uint8_t* qbuf = kbuf + p.stages * tile_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(qbuf + 2 * q_bytes);
+  // the current group's head weights, one copy per epilogue warp ([qi][h])
+  float* wbuf = reinterpret_cast<float*>(qbuf + 2 * q_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(wbuf + kEpiWarps * n_mma);
   uint64_t* empty = full + p.stages;
   uint64_t* acc_full = empty + p.stages;
   uint64_t* acc_empty = acc_full + 4;
@@ -292,6 +295,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         continue;
       }
+      // this warp's copy of the group's weights, read by broadcast below
+      float* wwarp = wbuf + (warp - 2) * n_mma;
+      if (g != wg_group) {
+        __syncwarp();
+        for (int i = lane; i < n_mma; i += 32) {
+          const int qi = i / p.Hi, t = t0 + qi;
+          wwarp[i] = t < p.Tq ? __ldg(p.idx_w + ((size_t)b * p.Tq + t) * p.Hi + (i - qi * p.Hi))
+                              : 0.0f;
+        }
+        __syncwarp();
+        wg_group = g;
+      }
       // the nq x Hi columns in pairs of 64-column chunks (one TMEM wait per
       // pair); each chunk's 64 head terms go to 8 independent partial sums
       // (integer-valued terms add exactly in any order)
@@ -311,11 +326,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           const int t = t0 + qi;
           if (t >= p.Tq) break;                 // warp-uniform
           const size_t row = (size_t)b * p.Tq + t;
-          const float4* w4 = reinterpret_cast<const float4*>(p.idx_w + row * p.Hi + h0);
+          const float4* w4 = reinterpret_cast<const float4*>(wwarp + qi * p.Hi + h0);
           float acc8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int i = 0; i < 64; i += 8) {
-            const float4 wa = __ldg(w4 + i / 4), wb = __ldg(w4 + i / 4 + 1);
+            const float4 wa = w4[i / 4], wb = w4[i / 4 + 1];
             acc8[0] = fmaf(wa.x, fmaxf(v[i], 0.0f), acc8[0]);
             acc8[1] = fmaf(wa.y, fmaxf(v[i + 1], 0.0f), acc8[1]);
             acc8[2] = fmaf(wa.z, fmaxf(v[i + 2], 0.0f), acc8[2]);
@@ -417,8 +432,8 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
   while (p.ncols < (uint32_t)(p.nacc * n_mma * p.sub)) p.ncols <<= 1;
   // key-tile ring: as deep as the shared memory left after the query
   // buffers, barriers and the group prefix allows (at most 6 or 8 stages)
-  const size_t fixed = 1024 + 2 * (size_t)n_mma * Di + (2 * 16 + 12) * sizeof(uint64_t) + 16 +
-                       (size_t)(p.G + 1 + 32) * sizeof(int);
+  const size_t fixed = 1024 + 2 * (size_t)n_mma * Di + (size_t)kEpiWarps * n_mma * sizeof(float) +
+                       (2 * 16 + 12) * sizeof(uint64_t) + 16 + (size_t)(p.G + 1 + 32) * sizeof(int);
   const size_t tile_bytes = (size_t)kTileM * p.sub * Di;
   const int max_stages = p.sub == 2 ? 6 : (n_mma <= 64 ? 8 : 5);
   p.stages = (int)std::min<size_t>(max_stages, (kSmemLimit - fixed) / tile_bytes);

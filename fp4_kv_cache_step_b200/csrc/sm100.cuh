@@ -138,16 +138,11 @@ __device__ __forceinline__ uint32_t cluster_addr(uint32_t saddr, uint32_t rank) 
   return r;
 }
 
-// This CTA's shared memory -> another CTA's shared memory in the cluster (no
-// multicast); completion as transaction bytes on the destination CTA's
-// mbarrier (`dst` and `bar` are shared::cluster addresses from cluster_addr).
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes,
-                                                  uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "r"(smem_u32(src)), "r"(bytes), "r"(bar)
-      : "memory");
+// 16-byte store into another CTA's shared memory (`addr` from cluster_addr).
+__device__ __forceinline__ void st_cluster128(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05

@@ -970,9 +970,11 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
 
 // Writes, in position order, every key above T and the first need_eq keys equal
 // to T (T = 0 selects every real key), then pads with -1 up to k.
-template <int KPT, int CS>
+// kBlk > 0: a kept block b is written as positions kBlk b .. kBlk b + kBlk - 1
+// (-1 from nv_pos on), and the padding covers kBlk slots per missing block.
+template <int KPT, int CS, int kBlk>
 __device__ void reg_emit(cg::cluster_group& cl, int rank, int pass, const uint32_t (&key)[KPT],
-                         int base, uint32_t T, int need_eq, int k, int n_valid,
+                         int base, uint32_t T, int need_eq, int k, int n_valid, int nv_pos,
                          const int32_t* crow, int32_t* out, RegShared& sc) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // (greater << 16 | equal) counts: a CTA's totals (at most 512 x 64) fit 16 bits each
@@ -1029,7 +1031,16 @@ __device__ void reg_emit(cg::cluster_group& cl, int rank, int pass, const uint32
       if (kk == T && kk != 0u) take = eq_seen++ < need_eq;
       if (take) {
         const int i = reg_pos<KPT>(base, j, q);
-        out[pos++] = crow ? __ldg(crow + i) : i;
+        if (kBlk) {
+#pragma unroll
+          for (int e = 0; e < kBlk; ++e) {
+            const int jj = i * kBlk + e;
+            out[(size_t)pos * kBlk + e] = jj < nv_pos ? jj : -1;
+          }
+          ++pos;
+        } else {
+          out[pos++] = crow ? __ldg(crow + i) : i;
+        }
       }
     }
     gt_run += (int)(tot >> 16);
@@ -1037,12 +1048,18 @@ __device__ void reg_emit(cg::cluster_group& cl, int rank, int pass, const uint32
   }
   if (rank == CS - 1) {
     const int total = min(k, n_valid);
-    for (int i = total + threadIdx.x; i < k; i += kRThreads) out[i] = -1;
+    const int per = kBlk ? kBlk : 1;
+    for (int i = total * per + threadIdx.x; i < k * per; i += kRThreads) out[i] = -1;
   }
   __syncthreads();
 }
 
-template <int KPT, int CS, bool kPool>
+// kBlk > 0 (blockwise pool): key slot b is block b, positions kBlk b ..
+// kBlk b + kBlk - 1 of the row, keyed by the largest score among its valid
+// positions (j < nvalid); a block with no valid position is not a candidate;
+// each kept block is written as its kBlk positions (-1 past nvalid), blocks
+// ascending, the pool -1 padded to K blocks.
+template <int KPT, int CS, bool kPool, int kBlk>
 __global__ void __launch_bounds__(kRThreads, 1)
 topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restrict__ nvalid,
                 const int32_t* __restrict__ cand, int K, int32_t* __restrict__ topk_out,
@@ -1060,7 +1077,9 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* srow = scores + row * ld;
   const int32_t* crow = kPool ? cand + row * ld : nullptr;
-  const int n = kPool ? ld : max(0, min(ld, nvalid[row]));
+  // candidates: valid positions, or blocks holding one
+  const int nv_pos = kPool ? ld : max(0, min(ld, nvalid[row]));
+  const int n = kBlk ? (nv_pos + kBlk - 1) / kBlk : nv_pos;
   // Whole rows of 16-byte aligned, 4-key-divisible length take branch-free
   // 16-byte loads (chunks past the row end read its first chunk, masked below),
   // so all of a thread's loads are in flight together; other rows load keys one
@@ -1069,7 +1088,38 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
                    ((reinterpret_cast<uintptr_t>(srow) | reinterpret_cast<uintptr_t>(crow)) & 15u) == 0;
   uint32_t key[KPT];
   int ids[kPool ? KPT : 1];
-  if (vec) {
+  if (kBlk) {
+    // each block's maximum over its valid positions (a NaN is kept, to be flagged)
+    const bool vec8 = kBlk % 4 == 0 && ld % 4 == 0 && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int b = reg_pos<KPT>(base, j / 4, j % 4);
+      float m = -INFINITY;
+      bool isnan_b = false;
+      if (b < n) {
+        const int j0 = b * kBlk;
+#pragma unroll
+        for (int e = 0; e < kBlk; e += 4) {
+          float v[4];
+          if (vec8 && j0 + e + 4 <= ld) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(srow + j0 + e));
+            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = (e + q < kBlk && j0 + e + q < ld) ? __ldg(srow + j0 + e + q) : 0.0f;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (e + q < kBlk && j0 + e + q < nv_pos) {
+              isnan_b |= v[q] != v[q];
+              m = fmaxf(m, v[q]);
+            }
+          }
+        }
+      }
+      key[j] = isnan_b ? 0x7fc00000u : __float_as_uint(m);
+    }
+  } else if (vec) {
 #pragma unroll
     for (int j = 0; j < KPT / 4; ++j) {
       const int p0 = reg_pos<KPT>(base, j, 0);
@@ -1173,40 +1223,75 @@ topk_reg_kernel(const float* __restrict__ scores, int ld, const int32_t* __restr
   for (int pass = 0; pass < 2; ++pass) {
     const int k = pass == 0 ? K : Cout;
     if (pass == 1 && cand_out == nullptr) break;
-    int32_t* out = pass == 0 ? topk_out + row * (size_t)K : cand_out + row * (size_t)Cout;
+    int32_t* out = pass == 0 ? topk_out + row * (size_t)K * (kBlk ? kBlk : 1)
+                             : cand_out + row * (size_t)Cout;
     uint32_t T = 0u;
     int need_eq = 0;
     if (n_valid > k)
       reg_threshold<KPT, CS>(cl, key, base, kmin, kmax, k, pass > 0, T, need_eq, sc);
-    reg_emit<KPT, CS>(cl, rank, pass, key, base, T, need_eq, k, n_valid, crow, out, sc);
+    reg_emit<KPT, CS, kBlk>(cl, rank, pass, key, base, T, need_eq, k, n_valid, nv_pos, crow, out,
+                            sc);
   }
   // Every access to another CTA's shared memory (the fine bins, the candidate
   // lists, and the values written into every CTA) precedes the last cluster
   // barrier in reg_emit, so a CTA may leave without waiting for the others.
 }
 
-template <int KPT, int CS>
+template <int KPT, int CS, int kBlk>
 cudaError_t launch_topk_reg(const float* scores, int ld, const int32_t* nvalid,
                             const int32_t* cand, int rows, int K, int32_t* topk_idx, int Cout,
                             int32_t* cand_out, int* err, cudaStream_t stream) {
   const dim3 grid((unsigned)(rows * CS)), cluster((unsigned)CS, 1, 1);
-  if (cand != nullptr)
-    return launch_pdl(topk_reg_kernel<KPT, CS, true>, grid, dim3(kRThreads), 0, stream, cluster,
-                      scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
-  return launch_pdl(topk_reg_kernel<KPT, CS, false>, grid, dim3(kRThreads), 0, stream, cluster,
-                    scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
+  if (cand != nullptr && kBlk == 0)
+    return launch_pdl(topk_reg_kernel<KPT, CS, true, 0>, grid, dim3(kRThreads), 0, stream,
+                      cluster, scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
+  return launch_pdl(topk_reg_kernel<KPT, CS, false, kBlk>, grid, dim3(kRThreads), 0, stream,
+                    cluster, scores, ld, nvalid, cand, K, topk_idx, Cout, cand_out, err);
 }
 
-template <int CS>
-cudaError_t launch_topk_reg_cs(const float* scores, int ld, const int32_t* nvalid,
+// `slots`: key slots per row (positions, or blocks in the block mode)
+template <int CS, int kBlk>
+cudaError_t launch_topk_reg_cs(const float* scores, int ld, int slots, const int32_t* nvalid,
                                const int32_t* cand, int rows, int K, int32_t* topk_idx, int Cout,
                                int32_t* cand_out, int* err, cudaStream_t stream) {
-  const int per = ceil_div(ceil_div(max(ld, 1), CS), kRThreads);
+  const int per = ceil_div(ceil_div(max(slots, 1), CS), kRThreads);
   if (per <= 4)
-    return launch_topk_reg<4, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+    return launch_topk_reg<4, CS, kBlk>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout,
+                                        cand_out, err, stream);
   if (per <= 16)
-    return launch_topk_reg<16, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
-  return launch_topk_reg<64, CS>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
+    return launch_topk_reg<16, CS, kBlk>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout,
+                                         cand_out, err, stream);
+  if constexpr (kBlk == 0)
+    return launch_topk_reg<64, CS, 0>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout,
+                                      cand_out, err, stream);
+  else
+    return cudaErrorInvalidValue;   // the block mode keeps at most 16 blocks per thread
+}
+
+// Cluster size for the register kernel: the largest of 1, 2, 4, 8 that keeps
+// rows x CS within the SMs.
+int reg_cluster_size(int rows, int sms) {
+  int rcs = 1;
+  while (rcs < 8 && rows * rcs * 2 <= sms) rcs *= 2;
+  return rcs;
+}
+
+template <int kBlk>
+cudaError_t launch_topk_reg_any(const float* scores, int ld, int slots, const int32_t* nvalid,
+                                const int32_t* cand, int rows, int K, int32_t* topk_idx,
+                                int Cout, int32_t* cand_out, int* err, cudaStream_t stream,
+                                int rcs) {
+  if (rcs == 8)
+    return launch_topk_reg_cs<8, kBlk>(scores, ld, slots, nvalid, cand, rows, K, topk_idx, Cout,
+                                       cand_out, err, stream);
+  if (rcs == 4)
+    return launch_topk_reg_cs<4, kBlk>(scores, ld, slots, nvalid, cand, rows, K, topk_idx, Cout,
+                                       cand_out, err, stream);
+  if (rcs == 2)
+    return launch_topk_reg_cs<2, kBlk>(scores, ld, slots, nvalid, cand, rows, K, topk_idx, Cout,
+                                       cand_out, err, stream);
+  return launch_topk_reg_cs<1, kBlk>(scores, ld, slots, nvalid, cand, rows, K, topk_idx, Cout,
+                                     cand_out, err, stream);
 }
 
 }  // namespace
@@ -1225,18 +1310,10 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
   // Register variant: a cluster of CS CTAs per row (as many as keep rows x CS
   // within the SMs), each holding at most 64 keys per thread in registers
   {
-    const int sms = topk_sm_count();
-    int rcs = 1;
-    while (rcs < 8 && rows * rcs * 2 <= sms) rcs *= 2;
-    if (ld <= rcs * kRThreads * 64) {
-      if (rcs == 8)
-        return launch_topk_reg_cs<8>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
-      if (rcs == 4)
-        return launch_topk_reg_cs<4>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
-      if (rcs == 2)
-        return launch_topk_reg_cs<2>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
-      return launch_topk_reg_cs<1>(scores, ld, nvalid, cand, rows, K, topk_idx, Cout, cand_out, err, stream);
-    }
+    const int rcs = reg_cluster_size(rows, topk_sm_count());
+    if (ld <= rcs * kRThreads * 64)
+      return launch_topk_reg_any<0>(scores, ld, ld, nvalid, cand, rows, K, topk_idx, Cout,
+                                    cand_out, err, stream, rcs);
   }
   // Few rows: a cluster of cs CTAs per row (cs = 2, 4 or 8, as many as keep
   // rows x cs within one wave), each staging a slice of the row.
@@ -1265,6 +1342,20 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
   }
   return launch_pdl(topk_kernel<false>, dim3(rows), dim3(kThreads), 0, stream, dim3(1), scores, ld,
                     nvalid, cand, K, topk_idx, Cout, cand_out, err);
+}
+
+// The blockwise pool in one launch of the register kernel (blocks of 8
+// positions); false when the shape is outside its range.
+bool launch_block_pool_reg(const float* scores, int ld, const int32_t* nvalid, int rows,
+                           int block, int nblocks, int32_t* cand, int* err, cudaStream_t stream,
+                           cudaError_t* e) {
+  if (block != 8 || rows == 0) return false;
+  const int nbmax = (ld + 7) / 8;
+  const int rcs = reg_cluster_size(rows, topk_sm_count());
+  if (nbmax > rcs * kRThreads * 16) return false;
+  *e = launch_topk_reg_any<8>(scores, ld, nbmax, nvalid, nullptr, rows, nblocks, cand, 0, nullptr,
+                              err, stream, rcs);
+  return true;
 }
 
 }  // namespace csa2
