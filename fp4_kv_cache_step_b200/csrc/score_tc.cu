@@ -60,6 +60,19 @@ __device__ __forceinline__ int group_tiles(const TcParams& p, int g) {
   return (nmax + rows - 1) / rows;
 }
 
+// Two fp32 fused multiply-adds as one packed instruction (each rounded once,
+// like fmaf).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t ua, ub, uc, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ua) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(ub) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(uc) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(ua), "l"(ub), "l"(uc));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+
 // The MMAs of one pipeline tile: SUB blocks of 128 entries x KSTEPS steps of
 // 32 key bytes. Descriptor start addresses advance by adding (bytes >> 4) to
 // the low field (shared-memory addresses stay below 2^18, so no carry).
@@ -75,10 +88,11 @@ __device__ __forceinline__ void issue_tile(uint32_t d0, uint64_t ad, uint64_t bd
                bd + (uint64_t)((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
 }
 
-// kDecode: one query per group with 64 indexer heads (the weights stay in
-// registers); otherwise the general epilogue, so that each path gets the
-// registers it needs.
-template <bool kDecode>
+// kHi indexer heads, kNq queries per group: (64, 1) is the decode path (the
+// weights stay in registers); otherwise the multi-query epilogue, with every
+// index constant, so that each shape gets the registers and instructions it
+// needs.
+template <int kHi, int kNq>
 __global__ void __launch_bounds__(kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap qmap, const TcParams p) {
@@ -104,6 +118,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   int* tile_pre = const_cast<int*>(reinterpret_cast<volatile int*>(tmem_slot + 2));   // [G + 1]
   int* scan_tmp = tile_pre + p.G + 1;                                               // [kThreads/32]
 
+  constexpr bool kDecode = kHi == 64 && kNq == 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait_and_release();
 
@@ -249,6 +264,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     int g = g_first, k = 0, wg_group = -1;
     float wreg[64];                            // head weights of the current query (nq == 1)
+    int nvq[kNq];                              // the group's query lengths (multi-query)
     int nv_cur = 0;
     for (int tile = lo; tile < hi; ++tile, ++k) {
       while (tile >= tile_pre[g + 1]) ++g;
@@ -295,60 +311,51 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         continue;
       }
-      // this warp's copy of the group's weights, read by broadcast below
-      float* wwarp = wbuf + (warp - 2) * n_mma;
+      // this warp's copy of the group's weights ([qi][h]), read by broadcast
+      // below, and the group's query lengths
+      float* wwarp = wbuf + (warp - 2) * (kNq * kHi);
       if (g != wg_group) {
         __syncwarp();
-        for (int i = lane; i < n_mma; i += 32) {
-          const int qi = i / p.Hi, t = t0 + qi;
-          wwarp[i] = t < p.Tq ? __ldg(p.idx_w + ((size_t)b * p.Tq + t) * p.Hi + (i - qi * p.Hi))
+#pragma unroll
+        for (int i = lane; i < kNq * kHi; i += 32) {
+          const int qi = i / kHi, t = t0 + qi;
+          wwarp[i] = t < p.Tq ? __ldg(p.idx_w + ((size_t)b * p.Tq + t) * kHi + (i - qi * kHi))
                               : 0.0f;
         }
+#pragma unroll
+        for (int qi = 0; qi < kNq; ++qi)
+          nvq[qi] = t0 + qi < p.Tq ? min(__ldg(p.nvalid + (size_t)b * p.Tq + t0 + qi), p.N) : 0;
         __syncwarp();
         wg_group = g;
       }
-      // the nq x Hi columns in pairs of 64-column chunks (one TMEM wait per
-      // pair); each chunk's 64 head terms go to 8 independent partial sums
+      // one 64-column chunk (64 heads of one query) at a time: ReLU, then the
+      // head weights by packed fp32 pairs into 4 partial sums per chunk
       // (integer-valued terms add exactly in any order)
-      const int nchunk = p.nq * (p.Hi / 64);
-      float part = 0.0f;                        // Hi = 128: the first half's sum
-      for (int c0 = 0; c0 < nchunk; c0 += 2) {
-        float va[64], vb[64];
-        const bool two = c0 + 1 < nchunk;
-        tmem_ld_64x2(acc_addr + (uint32_t)(c0 * 64), acc_addr + (uint32_t)((two ? c0 + 1 : c0) * 64),
-                     va, vb);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int c = c0 + half;
-          if (c >= nchunk) break;
-          const float* v = half ? vb : va;
-          const int qi = c / (p.Hi / 64), h0 = (c % (p.Hi / 64)) * 64;
-          const int t = t0 + qi;
-          if (t >= p.Tq) break;                 // warp-uniform
-          const size_t row = (size_t)b * p.Tq + t;
-          const float4* w4 = reinterpret_cast<const float4*>(wwarp + qi * p.Hi + h0);
-          float acc8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+      for (int qi = 0; qi < kNq; ++qi) {
+        float2 acc2[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                          make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+        for (int h0 = 0; h0 < kHi; h0 += 64) {
+          float v[64];
+          tmem_ld_64(acc_addr + (uint32_t)(qi * kHi + h0), v);
+          const float4* w4 = reinterpret_cast<const float4*>(wwarp + qi * kHi + h0);
 #pragma unroll
           for (int i = 0; i < 64; i += 8) {
             const float4 wa = w4[i / 4], wb = w4[i / 4 + 1];
-            acc8[0] = fmaf(wa.x, fmaxf(v[i], 0.0f), acc8[0]);
-            acc8[1] = fmaf(wa.y, fmaxf(v[i + 1], 0.0f), acc8[1]);
-            acc8[2] = fmaf(wa.z, fmaxf(v[i + 2], 0.0f), acc8[2]);
-            acc8[3] = fmaf(wa.w, fmaxf(v[i + 3], 0.0f), acc8[3]);
-            acc8[4] = fmaf(wb.x, fmaxf(v[i + 4], 0.0f), acc8[4]);
-            acc8[5] = fmaf(wb.y, fmaxf(v[i + 5], 0.0f), acc8[5]);
-            acc8[6] = fmaf(wb.z, fmaxf(v[i + 6], 0.0f), acc8[6]);
-            acc8[7] = fmaf(wb.w, fmaxf(v[i + 7], 0.0f), acc8[7]);
-          }
-          const float s = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) +
-                          ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-          float* dst = p.scores + row * p.N + j;
-          if (j < min(p.nvalid[row], p.N)) {
-            if (p.Hi == 64) *dst = s;
-            else if (h0 == 0) part = s;         // Hi = 128: two chunks per query
-            else *dst = part + s;
+            acc2[0] = ffma2(make_float2(wa.x, wa.y),
+                            make_float2(fmaxf(v[i], 0.0f), fmaxf(v[i + 1], 0.0f)), acc2[0]);
+            acc2[1] = ffma2(make_float2(wa.z, wa.w),
+                            make_float2(fmaxf(v[i + 2], 0.0f), fmaxf(v[i + 3], 0.0f)), acc2[1]);
+            acc2[2] = ffma2(make_float2(wb.x, wb.y),
+                            make_float2(fmaxf(v[i + 4], 0.0f), fmaxf(v[i + 5], 0.0f)), acc2[2]);
+            acc2[3] = ffma2(make_float2(wb.z, wb.w),
+                            make_float2(fmaxf(v[i + 6], 0.0f), fmaxf(v[i + 7], 0.0f)), acc2[3]);
           }
         }
+        const float sc = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) +
+                         ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
+        if (j < nvq[qi]) p.scores[((size_t)b * p.Tq + t0 + qi) * p.N + j] = sc;
       }
       tc_fence_before();
       __syncwarp();
@@ -449,9 +456,15 @@ cudaError_t launch_index_score_tc(const uint8_t* idx_q, const float* idx_w, cons
     return cudaErrorInvalidValue;
 
   const size_t smem = fixed + (size_t)p.stages * tile_bytes;
-  const bool dec = p.nq == 1 && Hi == 64;
-  void (*kernel)(CUtensorMap, CUtensorMap, TcParams) =
-      dec ? index_score_tc_kernel<true> : index_score_tc_kernel<false>;
+  void (*kernel)(CUtensorMap, CUtensorMap, TcParams) = nullptr;
+  if (Hi == 64) {
+    kernel = p.nq == 1   ? index_score_tc_kernel<64, 1>
+             : p.nq == 2 ? index_score_tc_kernel<64, 2>
+             : p.nq == 3 ? index_score_tc_kernel<64, 3>
+                         : index_score_tc_kernel<64, 4>;
+  } else {
+    kernel = p.nq == 1 ? index_score_tc_kernel<128, 1> : index_score_tc_kernel<128, 2>;
+  }
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

@@ -1031,7 +1031,24 @@ __device__ void reg_emit(cg::cluster_group& cl, int rank, int pass, const uint32
       if (kk == T && kk != 0u) take = eq_seen++ < need_eq;
       if (take) {
         const int i = reg_pos<KPT>(base, j, q);
-        if (kBlk) {
+        if (kBlk == 8) {
+          // the block's 8 positions as two 16-byte stores (rows and slots are
+          // 32-byte aligned)
+          const int j0 = i * 8;
+          int4 lo4, hi4;
+          lo4.x = j0 < nv_pos ? j0 : -1;
+          lo4.y = j0 + 1 < nv_pos ? j0 + 1 : -1;
+          lo4.z = j0 + 2 < nv_pos ? j0 + 2 : -1;
+          lo4.w = j0 + 3 < nv_pos ? j0 + 3 : -1;
+          hi4.x = j0 + 4 < nv_pos ? j0 + 4 : -1;
+          hi4.y = j0 + 5 < nv_pos ? j0 + 5 : -1;
+          hi4.z = j0 + 6 < nv_pos ? j0 + 6 : -1;
+          hi4.w = j0 + 7 < nv_pos ? j0 + 7 : -1;
+          int4* o4 = reinterpret_cast<int4*>(out + (size_t)pos * 8);
+          o4[0] = lo4;
+          o4[1] = hi4;
+          ++pos;
+        } else if (kBlk) {
 #pragma unroll
           for (int e = 0; e < kBlk; ++e) {
             const int jj = i * kBlk + e;
