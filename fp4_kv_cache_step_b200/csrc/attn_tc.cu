@@ -709,9 +709,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           ok = issue_s(next_s++);
           did = true;
         }
-        if (!did && (++spins & 63u) == 0u) {
-          __nanosleep(32);
-          if (*abort_flag || global_ns() - t0 > kWaitLimitNs) {
+        if (!did) {
+          // test_wait does not suspend: sleep between polls, so that this
+          // warp leaves its sub-partition's issue slots to the producer and
+          // softmax warps that share it
+          __nanosleep(40);
+          if ((++spins & 63u) == 0u && (*abort_flag || global_ns() - t0 > kWaitLimitNs)) {
             *abort_flag = 1;
             ok = false;
           }

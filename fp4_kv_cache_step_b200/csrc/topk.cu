@@ -745,9 +745,7 @@ constexpr int kRGroups = 64;                      // groups of 64 bins
 
 struct __align__(16) RegShared {
   int bins[kRBins];                 // this CTA's histogram (fine bins read by the cluster)
-  uint32_t cand_key[kRCandCap];     // this CTA's keys in the threshold bin (read by the cluster)
-  int cand_pos[kRCandCap];
-  uint32_t all_key[kRCandCap];      // the whole row's threshold bin
+  uint32_t all_key[kRCandCap];      // the whole row's threshold bin (written by every CTA)
   int all_pos[kRCandCap];
   // written by every CTA of the cluster into every CTA (slot = the writer's
   // rank), so that after a cluster barrier each CTA reads them locally
@@ -755,6 +753,7 @@ struct __align__(16) RegShared {
   uint32_t rng_min[8], rng_max[8];  // per rank: its key range and count of real keys
   int rng_cnt[8];
   uint32_t emit_from[2][8];         // per pass and rank: its (greater << 16 | equal) counts
+  int rank_cnt[8];                  // per rank: its keys in the threshold bin
   int warp_a[kRWarps], warp_b[kRWarps];
   uint32_t red_min[kRWarps], red_max[kRWarps];
   int bcast[8];
@@ -878,14 +877,22 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
       }
       const int fi = warp_incl_scan(f0 + f1);
       const int fb = fi - f0 - f1;
+      int win = -1;                                  // 0: bin top - 2 lane; 1: the next
       if (fb < kg && kg <= fb + f0) {
         sc.bcast[0] = top - 2 * lane;
         sc.bcast[1] = kg - fb;
         sc.bcast[2] = f0;
+        win = 0;
       } else if (fb + f0 < kg && kg <= fi) {
         sc.bcast[0] = top - 2 * lane - 1;
         sc.bcast[1] = kg - fb - f0;
         sc.bcast[2] = f1;
+        win = 1;
+      }
+      if (win >= 0) {
+        // every CTA's count of the threshold bin: the offsets of their candidates
+#pragma unroll
+        for (int r = 0; r < CS; ++r) sc.rank_cnt[r] = at_rank<CS>(cl, sc.bins, r)[top - 2 * lane - win];
       }
     }
     __syncthreads();
@@ -902,45 +909,32 @@ __device__ void reg_threshold(cg::cluster_group& cl, const uint32_t (&key)[KPT],
     }
     const uint32_t bw_m1 = (1u << shift) - 1u;
     if (cbin <= kRCandCap) {
-      // the keys of the threshold bin, from the whole cluster, ranked exactly
+      // the keys of the threshold bin, from the whole cluster, ranked exactly:
+      // each CTA writes its own into every CTA's list, at the offset given by
+      // the counts of the CTAs before it
+      int off = 0;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) off += r < rank ? sc.rank_cnt[r] : 0;
 #pragma unroll
       for (int j = 0; j < KPT; ++j) {
         const uint32_t kk = key[j];
         if (kk != 0u && kk >= lo && kk - lo <= bw_m1) {
-          const int slot = atomicAdd(&sc.ncand, 1);
+          const int slot = off + atomicAdd(&sc.ncand, 1);
           if (slot < kRCandCap) {
-            sc.cand_key[slot] = kk;
-            sc.cand_pos[slot] = reg_pos<KPT>(base, j / 4, j % 4);
+            const int pos = reg_pos<KPT>(base, j / 4, j % 4);
+#pragma unroll
+            for (int r = 0; r < CS; ++r) {
+              RegShared* o = at_rank<CS>(cl, &sc, r);
+              o->all_key[slot] = kk;
+              o->all_pos[slot] = pos;
+            }
           }
         }
       }
-      csync<CS>(cl);                               // every CTA's candidates are listed
-      int c;
-      const uint32_t* ck = sc.cand_key;
-      const int* cp = sc.cand_pos;
-      if (CS > 1) {
-        // every CTA's count first (independent loads), then one pass over all
-        int nr[CS], off[CS + 1];
-#pragma unroll
-        for (int r = 0; r < CS; ++r) nr[r] = min(at_rank<CS>(cl, &sc, r)->ncand, kRCandCap);
-        off[0] = 0;
-#pragma unroll
-        for (int r = 0; r < CS; ++r) off[r + 1] = off[r] + nr[r];
-        c = min(off[CS], kRCandCap);
-        for (int u = threadIdx.x; u < c; u += kRThreads) {
-          int r = 0;
-#pragma unroll
-          for (int q = 1; q < CS; ++q) r += u >= off[q];
-          const RegShared* o = at_rank<CS>(cl, &sc, r);
-          sc.all_key[u] = o->cand_key[u - off[r]];
-          sc.all_pos[u] = o->cand_pos[u - off[r]];
-        }
-        ck = sc.all_key;
-        cp = sc.all_pos;
-        __syncthreads();
-      } else {
-        c = min(sc.ncand, kRCandCap);
-      }
+      csync<CS>(cl);                               // every CTA's candidates are everywhere
+      const int c = min(cbin, kRCandCap);
+      const uint32_t* ck = sc.all_key;
+      const int* cp = sc.all_pos;
       for (int u = threadIdx.x; u < c; u += kRThreads) {
         const uint32_t ku = ck[u];
         const int pu = cp[u];
