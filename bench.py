@@ -62,9 +62,9 @@ KERNEL_SOURCES = {
 # the kernels' names as ncu lists them (regular expressions)
 KERNEL_NAMES = {
     "score": r"index_score",
-    "topk": r"topk_(reg_|cluster_)?kernel",
+    "topk": r"topk_reg_kernel<\d+, \d+, [01], 0>|topk_cluster_kernel|topk_kernel<",
     "attn": r"sparse_attn_tc_kernel",
-    "block_pool": r"block_(max|expand)_kernel",
+    "block_pool": r"topk_reg_kernel<\d+, \d+, [01], 8>|block_(max|expand)_kernel",
 }
 
 
