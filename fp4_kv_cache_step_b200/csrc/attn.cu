@@ -57,6 +57,7 @@ attn_combine_kernel(const float* __restrict__ ws_o, const float2* __restrict__ w
 
 struct SplitPlan {
   int nhb, nsplit, split_len;
+  bool cluster;   // up to the largest cluster, the splits may merge inside a cluster
 };
 
 int sm_count() {
@@ -83,6 +84,15 @@ SplitPlan plan_splits(int rows, int Hq, int K) {
   if (nsplit > cmax && nsplit < 2 * cmax) nsplit = cmax;
   nsplit = min(nsplit, ceil_div(K, tile));
   nsplit = max(nsplit, 1);
+  // ... as long as all of the clusters are resident at once: where they would
+  // need a second wave, the splits go through the workspace and the combine
+  // kernel instead, one wave of as many splits as the SMs allow
+  p.cluster = true;
+  if (nsplit > 1 && nsplit <= cmax && sparse_attn_tc_cluster_capacity(nsplit) < ctas) {
+    nsplit = ctas >= sms ? 1 : sms / ctas;
+    nsplit = max(1, min(nsplit, ceil_div(K, tile)));
+    p.cluster = false;
+  }
   p.split_len = ceil_div(ceil_div(K, nsplit), tile) * tile;
   p.nsplit = ceil_div(K, p.split_len);
   return p;
@@ -117,7 +127,8 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
   bool merged = false;
   cudaError_t e = launch_sparse_attn_tc(q, kv_packed, kv_scale, topk_idx, rows, Tq, Hq, N, K,
                                         softmax_scale, p.nhb, p.nsplit, p.split_len, out, lse,
-                                        ws_o, ws_ml, err, stream, &merged, swa);
+                                        ws_o, ws_ml, err, stream, p.cluster ? &merged : nullptr,
+                                        swa);
   if (e != cudaSuccess || p.nsplit == 1 || merged) return e;
   return launch_pdl(attn_combine_kernel, dim3(rows, Hq), dim3(128), 0, stream, dim3(1), ws_o,
                     ws_ml, Hq, p.nhb, p.nsplit, out, lse);

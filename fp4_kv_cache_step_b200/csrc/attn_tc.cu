@@ -992,10 +992,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
 
 template <bool kG16>
 struct KernelSetup {
-  // cudaFuncSetAttribute and the cluster occupancy query, once per device
-  static cudaError_t prepare(bool* clusters_ok) {
+  // cudaFuncSetAttribute and the cluster occupancy queries (how many clusters
+  // of each size 2 .. kMaxClusterSplits can be resident at once), once per
+  // device
+  static cudaError_t prepare(bool* clusters_ok, int* capacity = nullptr) {
     static int done[64] = {};
-    static int cluster_fit[64] = {};
+    static int cap[64][kMaxClusterSplits + 1] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1004,25 +1006,28 @@ struct KernelSetup {
       e = cudaFuncSetAttribute(sparse_attn_tc_kernel<kG16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
       if (e != cudaSuccess) return e;
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kMaxClusterSplits, 1, kMaxClusterSplits);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = kSmemBytes;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 1;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = kMaxClusterSplits;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      cluster_fit[dev] = cudaOccupancyMaxActiveClusters(&n, sparse_attn_tc_kernel<kG16>, &cfg) ==
-                                 cudaSuccess &&
-                             n > 0;
-      (void)cudaGetLastError();
+      for (int cs = 2; cs <= kMaxClusterSplits; ++cs) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kMaxClusterSplits, 1, (unsigned)cs);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = (unsigned)cs;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        cap[dev][cs] = cudaOccupancyMaxActiveClusters(&n, sparse_attn_tc_kernel<kG16>, &cfg) ==
+                               cudaSuccess ? n : 0;
+        (void)cudaGetLastError();
+      }
       done[dev] = 1;
     }
-    *clusters_ok = cluster_fit[dev] != 0;
+    *clusters_ok = cap[dev][kMaxClusterSplits] > 0;
+    if (capacity)
+      for (int cs = 0; cs <= kMaxClusterSplits; ++cs) capacity[cs] = cs < 2 ? 0 : cap[dev][cs];
     return cudaSuccess;
   }
 };
@@ -1031,6 +1036,15 @@ struct KernelSetup {
 
 int sparse_attn_tc_tile() { return kT; }
 int sparse_attn_tc_max_cluster() { return kMaxClusterSplits; }
+
+int sparse_attn_tc_cluster_capacity(int cs) {
+  if (cs < 2 || cs > kMaxClusterSplits) return 0;
+  bool ok = false;
+  int cap[kMaxClusterSplits + 1];
+  // with no device to ask, assume one wave of clusters fits (host-side sizing)
+  if (KernelSetup<false>::prepare(&ok, cap) != cudaSuccess) return 1 << 20;
+  return cap[cs];
+}
 
 cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,

@@ -155,6 +155,9 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
 // ws_o/ws_ml for attn_combine_kernel.
 int sparse_attn_tc_tile();
 int sparse_attn_tc_max_cluster();   // splits of a row that merge inside one cluster
+// how many clusters of `cs` splits can be resident at once on the current
+// device (a large number when no device can be asked)
+int sparse_attn_tc_cluster_capacity(int cs);
 cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   const uint8_t* kv_scale, const int32_t* topk_idx, int rows,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
