@@ -1321,7 +1321,10 @@ cudaError_t launch_topk(const float* scores, int ld, const int32_t* nvalid, cons
   // Register variant: a cluster of CS CTAs per row (as many as keep rows x CS
   // within the SMs), each holding at most 64 keys per thread in registers
   {
-    const int rcs = reg_cluster_size(rows, topk_sm_count());
+    int rcs = reg_cluster_size(rows, topk_sm_count());
+    // rows too long for that many CTAs: the smallest cluster that holds them,
+    // in more than one wave (still far ahead of the shared-memory kernels)
+    while (rcs < 8 && ld > rcs * kRThreads * 64) rcs *= 2;
     if (ld <= rcs * kRThreads * 64)
       return launch_topk_reg_any<0>(scores, ld, ld, nvalid, cand, rows, K, topk_idx, Cout,
                                     cand_out, err, stream, rcs);
