@@ -499,7 +499,10 @@ csa2_status csa2_layer_step(const csa2_layer_args* a, csa2_mode mode, csa2_share
   e = csa2::launch_sparse_attn(a->q, st->kv_packed, st->kv_scale, st->topk_idx, a->B, a->Tq, a->Hq,
                                a->N, a->K, a->softmax_scale, a->out, a->lse,
                                ws ? ws + scores_bytes + pool_bytes : nullptr, err, cs,
-                               a->swa_kv ? &win : nullptr);
+                               a->swa_kv ? &win : nullptr,
+                               // FULL / REINDEX: two kernels of this call precede
+                               // the attention, so the caller's query is complete
+                               mode != CSA2_MODE_REUSE);
   if (e != cudaSuccess) return cuda_fail(e, "csa2_layer_step attention");
   return ok();
 }

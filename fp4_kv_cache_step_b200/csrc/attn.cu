@@ -112,7 +112,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
                                float* lse, void* workspace, int* err, cudaStream_t stream,
-                               const SwaWindow* swa) {
+                               const SwaWindow* swa, bool q_ready) {
   const int rows = B * Tq;
   if (rows == 0) return cudaSuccess;
   // the window's entries follow the selected ones in each row's entry list
@@ -128,7 +128,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
   cudaError_t e = launch_sparse_attn_tc(q, kv_packed, kv_scale, topk_idx, rows, Tq, Hq, N, K,
                                         softmax_scale, p.nhb, p.nsplit, p.split_len, out, lse,
                                         ws_o, ws_ml, err, stream, p.cluster ? &merged : nullptr,
-                                        swa);
+                                        swa, q_ready);
   if (e != cudaSuccess || p.nsplit == 1 || merged) return e;
   return launch_pdl(attn_combine_kernel, dim3(rows, Hq), dim3(128), 0, stream, dim3(1), ws_o,
                     ws_ml, Hq, p.nhb, p.nsplit, out, lse);

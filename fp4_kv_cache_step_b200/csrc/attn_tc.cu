@@ -32,8 +32,8 @@
 // conversions and one fp16 product per value. A producer dequantises a tile into
 // registers BEFORE waiting for its ring slot, so after the slot frees only the
 // shared-memory stores stand between P(t-3) V(t-3) and S(t).
-// Roles: warps 0-7 gather and dequantise, and stage Q into tensor memory after
-// the first tile; warp 8 owns tensor memory and issues the MMAs; warps 9-12 run
+// Roles: warps 0-7 gather and dequantise, and stage Q into tensor memory while
+// the first tile's rows are in flight; warp 8 owns tensor memory and issues the MMAs; warps 9-12 run
 // the softmax. At the
 // end every warp that can reach a quadrant's O lanes (its softmax warp and two
 // producer warps) writes that quadrant's output, partial or final. Every
@@ -280,6 +280,7 @@ struct AttnParams {
   float2* ws_ml;
   int* err;
   int cluster_merge;   // the splits of a (row, head block) form a cluster and merge in DSMEM
+  int q_before_wait;   // the query may be read before the wait for the preceding kernel
 };
 
 // Raw bytes a producer lane holds for one entry: the codes (8 B) and scales
@@ -345,14 +346,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     }
     sm.abort_flag = 0;
     fence_mbar_init();
+    // the block's query rows (1 KB each, contiguous) into V slot 2 in one bulk
+    // copy: before the wait for the preceding kernel when the caller vouches
+    // that the query was complete before it (the layer step: it comes from
+    // before the scorer, two kernels back)
+    if (p.q_before_wait) {
+      const uint32_t qbytes = (uint32_t)nh * kD * 2;
+      mbar_arrive_expect_tx(&sm.bar.q_ld, qbytes);
+      bulk_load(vs + 2 * kVTile, p.q + ((row * p.Hq) + h0) * kD, qbytes, &sm.bar.q_ld);
+    }
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_slot, kTmemCols);
   pdl_wait_and_release();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x == 0) {
-    // the block's query rows (1 KB each, contiguous) into V slot 2 in one bulk copy
+  if (threadIdx.x == 0 && !p.q_before_wait) {
     const uint32_t qbytes = (uint32_t)nh * kD * 2;
     mbar_arrive_expect_tx(&sm.bar.q_ld, qbytes);
     bulk_load(vs + 2 * kVTile, p.q + ((row * p.Hq) + h0) * kD, qbytes, &sm.bar.q_ld);
@@ -510,8 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     // c ^ (hh & 7). A row's largest magnitude is taken on the bf16 bit patterns
     // (non-negative floats order like their bits) with one warp reduction. Then
     // thread (h, ch) of warp w moves dims 256 ch + 128 (w / 4) .. + 127 of row h
-    // into tensor memory. This runs after the first tile is published and
-    // overlaps the second tile's loads.
+    // into tensor memory. This overlaps the first tile's row loads.
     auto stage_q = [&]() {
       const uint32_t qsm = vs_s + 2 * kVTile;
       bool ok = mbar_wait_warp(&sm.bar.q_ld, 0, abort_flag);
@@ -613,9 +621,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
     Raw ra[2], rb[2];
     load_half(id_cur, ra, 0);
     load_half(id_cur, rb, 1);
-    // the query block is staged after the first tile (slot 0) is published, so
-    // its conversion overlaps the loads of the second; every split has a tile
-    if (nt == 0) stage_q();
+    // the query block is staged while the first tile's rows are in flight
+    stage_q();
     for (int t = 0; t < nt; ++t) {
       const int buf = t % kRing;
       uint4 dq[2][4];
@@ -635,7 +642,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.bar.v_full[buf]);
-      if (t == 0) stage_q();
       const int id_far_checked = check_index(id_far, t + 3);
       prefetch_rows(id_far_checked);
       id_far = fetch_index(t + 4);
@@ -1051,7 +1057,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
                                   float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
-                                  bool* merged, const SwaWindow* swa) {
+                                  bool* merged, const SwaWindow* swa, bool q_ready) {
   AttnParams p;
   p.q = q;
   p.kv_packed = kv_packed;
@@ -1076,6 +1082,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
   p.ws_ml = ws_ml;
   p.err = err;
   p.cluster_merge = 0;
+  p.q_before_wait = q_ready ? 1 : 0;
   // no block-scale array: rows of the 16-channel layout
   const bool g16 = kv_scale == nullptr;
   void (*kernel)(AttnParams) = g16 ? sparse_attn_tc_kernel<true> : sparse_attn_tc_kernel<false>;

@@ -141,13 +141,15 @@ bool launch_block_pool_reg(const float* scores, int ld, const int32_t* nvalid, i
 // Sparse attention; see csa2_sparse_attn. With kv_scale NULL, kv_packed holds
 // the 16-channel layout (csa2_sparse_attn_g16): per entry D/2 code bytes then
 // D/16 E4M3 scale bytes. With swa non-null the window branch joins the same
-// softmax; the workspace is then sized for K + swa->W entries.
+// softmax; the workspace is then sized for K + swa->W entries. q_ready: the
+// query was complete before the kernel that precedes this one on the stream
+// started, so it may be read before the wait for that kernel.
 size_t sparse_attn_workspace_bytes(int B, int Tq, int Hq, int K);
 cudaError_t launch_sparse_attn(const uint16_t* q, const uint8_t* kv_packed,
                                const uint8_t* kv_scale, const int32_t* topk_idx, int B, int Tq,
                                int Hq, int N, int K, float softmax_scale, uint16_t* out,
                                float* lse, void* workspace, int* err, cudaStream_t stream,
-                               const SwaWindow* swa = nullptr);
+                               const SwaWindow* swa = nullptr, bool q_ready = false);
 
 // Tensor-core attention kernel (attn_tc.cu). With nsplit > 1 the splits are
 // merged inside the kernel (thread-block clusters, *merged set to true) when
@@ -163,6 +165,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t* q, const uint8_t* kv_packed,
                                   int Tq, int Hq, int N, int K, float softmax_scale, int nhb,
                                   int nsplit, int split_len, uint16_t* out, float* lse,
                                   float* ws_o, float2* ws_ml, int* err, cudaStream_t stream,
-                                  bool* merged, const SwaWindow* swa = nullptr);
+                                  bool* merged, const SwaWindow* swa = nullptr,
+                                  bool q_ready = false);
 
 }  // namespace csa2
