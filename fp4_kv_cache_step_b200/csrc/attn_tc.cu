@@ -944,41 +944,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
       return r == split ? reinterpret_cast<const float2*>(vs + kMergeSendMlOff + split * mlb)[i]
                         : reinterpret_cast<const float2*>(vs + kMergeRecvMlOff + r * mlb)[i];
     };
-    // one 16-byte chunk (8 dims) of one head per unit; every split's (max, sum)
-    // and chunk are loaded first, then the weights and the sum
+    // one 16-byte chunk (8 dims) of one head per unit, in a compact loop over
+    // the splits (this code runs once per CTA: its size, not its issue rate,
+    // decides its time)
     const int units = got ? nhm * (kD / 8) : 0;
 #pragma unroll 1
     for (int uo = threadIdx.x; uo < units; uo += kThreads) {
       const int i = uo / (kD / 8), cl16 = uo % (kD / 8);
       const int off = (cl16 ^ (i & 7)) << 4;
-      float2 ml[kMaxClusterSplits];
-      uint4 v[kMaxClusterSplits];
-#pragma unroll
-      for (int r = 0; r < kMaxClusterSplits; ++r) {
-        if (r < ns) {
-          ml[r] = part_ml(r, i);
-          v[r] = lds128(part_row(r, i) + off);
-        } else {
-          ml[r] = make_float2(-INFINITY, 0.0f);
-          v[r] = make_uint4(0, 0, 0, 0);
-        }
-      }
       float M = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < kMaxClusterSplits; ++r) M = fmaxf(M, ml[r].x);
-      float w[kMaxClusterSplits];
+#pragma unroll 1
+      for (int r = 0; r < ns; ++r) M = fmaxf(M, part_ml(r, i).x);
       float L = 0.0f;
-#pragma unroll
-      for (int r = 0; r < kMaxClusterSplits; ++r) {
-        w[r] = (ml[r].x != -INFINITY && ml[r].y > 0.0f) ? fast_exp2(ml[r].x - M) * ml[r].y : 0.0f;
-        L += w[r];
-      }
-      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
       float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-      for (int r = 0; r < kMaxClusterSplits; ++r) {
-        const float wr = w[r] * inv;
-        const uint32_t vw[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll 1
+      for (int r = 0; r < ns; ++r) {
+        const float2 ml = part_ml(r, i);
+        const float wr = (ml.x != -INFINITY && ml.y > 0.0f) ? fast_exp2(ml.x - M) * ml.y : 0.0f;
+        L += wr;
+        const uint4 v = lds128(part_row(r, i) + off);
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&vw[k]));
@@ -986,6 +971,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_tc_kernel(const AttnP
           acc[2 * k + 1] = fmaf(wr, f2.y, acc[2 * k + 1]);
         }
       }
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] *= inv;
       *reinterpret_cast<uint4*>(p.out + ((row * p.Hq) + h0 + hA + i) * kD + 8 * cl16) =
           make_uint4(pack_bf162(acc[0], acc[1]), pack_bf162(acc[2], acc[3]),
                      pack_bf162(acc[4], acc[5]), pack_bf162(acc[6], acc[7]));
