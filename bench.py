@@ -133,12 +133,14 @@ def profiled_traffic(kernel: str, workload: str, units: float):
             continue
         if r.get("workload") == workload:
             return float(r["dram_bytes_per_launch"]), "ncu capture of this workload"
-        best = best or r
-    if best is not None and best.get("units"):
+        if best is None and r.get("units"):
+            best = r                     # the first capture that can be scaled
+    if best is not None:
         return float(best["dram_bytes_per_launch"]) * units / float(best["units"]), \
             "ncu capture of %s scaled by units (%s)" % (best["workload"], best.get("unit_kind"))
     if any(r.get("kernel") == kernel and r.get("sources_sha1") == sha for r in recs):
-        return None, "no ncu capture of this workload (the kernel's other captures carry no unit count to scale by)"
+        return None, ("no ncu capture of this workload (the kernel's other captures carry "
+                      "no unit count to scale by)")
     return None, "sources changed since the last ncu capture"
 
 
